@@ -1,0 +1,253 @@
+"""Plain fp64 CPU oracle for Heavily Compressed Attention (HCA).
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import, call or
+execute this module: only the tests, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` use it.  It shares
+no code with the CUDA library; it is deliberately slow and written so that each
+step can be checked against the pages by eye.
+
+What the pages say (all prose, no equations):
+
+* 'BaiduがERNIE 5.5 Flash Baseを公開' (hackernews.jp), §2.1 Latent-Gated Sparse
+  Attention, and its Chinese twin 'ERNIE 5.5 Flash Base 正式发布' §2.1: an HCA
+  layer turns every 128 tokens into one cache entry and runs dense attention
+  over all of those entries plus a short window of recent uncompressed tokens;
+  HCA heads are 512 wide for query/key and value; the model has 64 attention
+  heads; every layer multiplies its attention output by a learned gate.
+* xenospectrum, 'ERNIE 5.5 Flash Base' analysis, section 活性140億パラメータと
+  長文処理を支える仕組み: the window is the most recent 128 tokens, kept
+  uncompressed as a sliding window.
+
+Readings adopted where the pages are silent (each is listed with its reason in
+the design notes of the repository):
+
+* one shared KV head; the compressor of block j is the within-block
+  softmax(s)-weighted sum of the block's K rows and, with the same weights, of
+  its V rows, where s is a per-token scalar score input;
+* query t sees compressed entry j only if block j lies wholly before its
+  window, i.e. j < nc(t) = max(0, floor((t - W + 1) / blk)), and the raw keys
+  max(0, t - W + 1) .. t (the window includes the query token itself);
+* one softmax over the union of both key sets, one scale 1/sqrt(D) for all
+  keys, no positional encoding, no sink;
+* out = sigmoid(g) * o, elementwise over [T, H, D].
+
+Parity status: pinned.  The tests under ``tests/test_oracle_pins.py`` tie
+every function here to something other than itself: a brute-force loop
+implementation with an explicitly built key list and mask; PyTorch's fp64
+``scaled_dot_product_attention`` for the cases that reduce to causal and
+banded attention; closed forms (constant block, uniform scores, gate at 0,
+hand-derived golden values); invariants (shift, permutation); and decode vs
+prefill agreement.
+"""
+from __future__ import annotations
+
+import math
+from typing import Iterable, Optional, Sequence
+
+import numpy as np
+
+HEADS = 64
+HEAD_DIM = 512
+BLOCK = 128
+WINDOW = 128
+
+
+# ---------------------------------------------------------------------------
+# Visibility rule
+# ---------------------------------------------------------------------------
+def window_start(t: int, win: int = WINDOW) -> int:
+    """First raw key of query t's window: the last `win` tokens up to and
+    including t (xenospectrum analysis, 活性140億パラメータと長文処理を支える
+    仕組み: the newest 128 tokens stay uncompressed)."""
+    return max(0, t - win + 1)
+
+
+def num_visible_blocks(t: int, blk: int = BLOCK, win: int = WINDOW) -> int:
+    """nc(t): how many compressed entries query t sees.
+
+    Block j covers tokens blk*j .. blk*j + blk - 1.  It is visible when it lies
+    wholly before the window, i.e. blk*(j+1) <= t - win + 1.  Counting the j
+    that satisfy this gives floor((t - win + 1) / blk), clamped at 0.
+    ('BaiduがERNIE 5.5 Flash Baseを公開' §2.1: entries for every 128 tokens,
+    plus a short raw window.)
+    """
+    return max(0, (t - win + 1) // blk)
+
+
+# ---------------------------------------------------------------------------
+# Compressor
+# ---------------------------------------------------------------------------
+def block_weights(s_block: np.ndarray) -> np.ndarray:
+    """softmax over the tokens of one block (last axis), max-subtracted."""
+    z = s_block - s_block.max(axis=-1, keepdims=True)
+    e = np.exp(z)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def compress(k: np.ndarray, v: np.ndarray, s: np.ndarray, blk: int = BLOCK):
+    """Compressed cache entries for every complete block.
+
+    k, v: [B, T, D]; s: [B, T].  Returns cK, cV: [B, T // blk, D] in fp64.
+    Entry j = sum_i softmax(s[blk*j : blk*j+blk])_i * row_i.  Tokens of a
+    trailing partial block are not compressed.
+    ('BaiduがERNIE 5.5 Flash Baseを公開' §2.1: 128 tokens -> 1 cache entry.)
+    """
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    s = np.asarray(s, dtype=np.float64)
+    B, T, D = k.shape
+    nb = T // blk
+    kb = k[:, : nb * blk].reshape(B, nb, blk, D)
+    vb = v[:, : nb * blk].reshape(B, nb, blk, D)
+    w = block_weights(s[:, : nb * blk].reshape(B, nb, blk))
+    ck = np.einsum("bni,bnid->bnd", w, kb)
+    cv = np.einsum("bni,bnid->bnd", w, vb)
+    return ck, cv
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round fp64 values to the nearest bfloat16 (ties to even), returned as
+    fp64.  Used only by the optional diagnosis mode that mimics a bf16 cache."""
+    f32 = np.asarray(x, dtype=np.float32)
+    bits = f32.view(np.uint32).astype(np.uint64)
+    lsb = (bits >> 16) & 1
+    rounded = ((bits + 0x7FFF + lsb) >> 16) << 16
+    out = rounded.astype(np.uint32).view(np.float32)
+    nan = np.isnan(f32)
+    out = np.where(nan, f32, out)
+    return out.astype(np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Attention core
+# ---------------------------------------------------------------------------
+def sigmoid(x: np.ndarray) -> np.ndarray:
+    return 1.0 / (1.0 + np.exp(-x))
+
+
+def attend(qrows: np.ndarray, keys: np.ndarray, values: np.ndarray,
+           mask: np.ndarray, scale: float):
+    """Dense masked softmax attention, all heads sharing one key/value set.
+
+    qrows: [n, H, D]; keys, values: [K, D]; mask: [n, K] (True = visible).
+    Returns o: [n, H, D] (normalised, ungated) and lse: [n, H] (natural log of
+    the softmax denominator of the scaled scores).
+    """
+    z = np.einsum("nhd,kd->nhk", qrows, keys) * scale
+    z = np.where(mask[:, None, :], z, -np.inf)
+    m = z.max(axis=-1, keepdims=True)
+    e = np.exp(z - m)
+    den = e.sum(axis=-1, keepdims=True)
+    o = np.einsum("nhk,kd->nhd", e / den, values)
+    lse = (m + np.log(den))[..., 0]
+    return o, lse
+
+
+def _prefill_rows(qb, gb, kb, vb, ckb, cvb, positions: np.ndarray,
+                  blk: int, win: int, scale: float):
+    """Outputs for the given query positions of one sequence.
+
+    The key set is the union over these positions: the compressed entries
+    0 .. max nc - 1 and the raw tokens from the earliest window start to the
+    last position; the per-row mask then selects each query's own keys.
+    """
+    t_lo, t_hi = int(positions.min()), int(positions.max())
+    n_c = num_visible_blocks(t_hi, blk, win)
+    r0 = window_start(t_lo, win)
+    keys = np.concatenate([ckb[:n_c], kb[r0 : t_hi + 1]], axis=0)
+    vals = np.concatenate([cvb[:n_c], vb[r0 : t_hi + 1]], axis=0)
+    raw_idx = np.arange(r0, t_hi + 1)
+    ent_idx = np.arange(n_c)
+    mask = np.zeros((len(positions), n_c + len(raw_idx)), dtype=bool)
+    for row, t in enumerate(positions):
+        t = int(t)
+        mask[row, :n_c] = ent_idx < num_visible_blocks(t, blk, win)
+        mask[row, n_c:] = (raw_idx >= window_start(t, win)) & (raw_idx <= t)
+    o, lse = attend(qb[positions], keys, vals, mask, scale)
+    out = sigmoid(gb[positions]) * o
+    return out, lse
+
+
+def prefill_forward(q, k, v, s, g, blk: int = BLOCK, win: int = WINDOW,
+                    scale: Optional[float] = None,
+                    positions: Optional[Sequence[int]] = None,
+                    round_cache_bf16: bool = False, chunk: int = 128,
+                    return_lse: bool = False, cache=None):
+    """HCA prefill forward in fp64.
+
+    q, g: [B, T, H, D]; k, v: [B, T, D]; s: [B, T].  Returns out [B, T, H, D]
+    (or [B, len(positions), H, D] when `positions` selects rows), and the lse
+    [.., H] when asked.  `cache` may pass precomputed (cK, cV) from
+    ``compress`` to avoid recomputing them.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    g = np.asarray(g, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, T, H, D = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    ck, cv = cache if cache is not None else compress(k, v, s, blk)
+    if round_cache_bf16:
+        ck, cv = round_bf16(ck), round_bf16(cv)
+    pos = np.arange(T) if positions is None else np.asarray(list(positions), dtype=np.int64)
+    out = np.empty((B, len(pos), H, D), dtype=np.float64)
+    lse = np.empty((B, len(pos), H), dtype=np.float64)
+    for b in range(B):
+        for c0 in range(0, len(pos), chunk):
+            sel = pos[c0 : c0 + chunk]
+            o, l = _prefill_rows(q[b], g[b], k[b], v[b], ck[b], cv[b], sel, blk, win, scale)
+            out[b, c0 : c0 + chunk] = o
+            lse[b, c0 : c0 + chunk] = l
+    return (out, lse) if return_lse else out
+
+
+def decode_forward(q, ck, cv, wk, wv, ctx_len, g, blk: int = BLOCK,
+                   win: int = WINDOW, scale: Optional[float] = None,
+                   return_lse: bool = False):
+    """HCA decode for one new token per sequence, in fp64.
+
+    q, g: [S, H, D]; ck, cv: [S, max_nc, D]; wk, wv: [S, win, D] hold the
+    window as a ring, the token at position p in slot p mod win; ctx_len[s] = L
+    counts the new token, so the query sits at t = L - 1.  Keys are the
+    compressed entries j < nc(L - 1) and the min(L, win) newest raw tokens
+    (slots 0 .. L-1 when L < win, all slots otherwise).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    g = np.asarray(g, dtype=np.float64)
+    ck = np.asarray(ck, dtype=np.float64)
+    cv = np.asarray(cv, dtype=np.float64)
+    wk = np.asarray(wk, dtype=np.float64)
+    wv = np.asarray(wv, dtype=np.float64)
+    S, H, D = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    out = np.empty((S, H, D), dtype=np.float64)
+    lse = np.empty((S, H), dtype=np.float64)
+    for si in range(S):
+        L = int(ctx_len[si])
+        t = L - 1
+        n_c = num_visible_blocks(t, blk, win)
+        n_w = min(L, win)
+        keys = np.concatenate([ck[si, :n_c], wk[si, :n_w]], axis=0)
+        vals = np.concatenate([cv[si, :n_c], wv[si, :n_w]], axis=0)
+        mask = np.ones((1, keys.shape[0]), dtype=bool)
+        o, l = attend(q[si][None], keys, vals, mask, scale)
+        out[si] = sigmoid(g[si]) * o[0]
+        lse[si] = l[0]
+    return (out, lse) if return_lse else out
+
+
+# ---------------------------------------------------------------------------
+# Work counts (used for FLOP accounting and by the tests)
+# ---------------------------------------------------------------------------
+def visited_pairs(T: int, blk: int = BLOCK, win: int = WINDOW) -> int:
+    """Number of (query, key) pairs one head visits over a sequence of T
+    tokens: sum over t of nc(t) + min(t + 1, win)."""
+    return sum(num_visible_blocks(t, blk, win) + (t - window_start(t, win) + 1)
+               for t in range(T))
+
+
+def decode_keys(ctx_len: Iterable[int], blk: int = BLOCK, win: int = WINDOW) -> int:
+    """Keys visited by one decode call: sum over sequences of nc(L-1) + min(L, win)."""
+    return sum(num_visible_blocks(int(L) - 1, blk, win) + min(int(L), win) for L in ctx_len)
