@@ -1,0 +1,507 @@
+#!/usr/bin/env python
+"""Benchmark of the HCA forward hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--quick]
+
+One step = one pass of the prefill hot path over the 32K-token workload
+(B = 1, T = 32768, 64 query heads x 512, one KV head, K scaled by 0.5):
+hca_compress (256 blocks) followed by hca_prefill_fwd with the gate fused.
+Inputs are resident in HBM and larger than L2 (4.3 GB per step).  The value is
+prefill TFLOP/s counting 4 * 64 * 512 FLOPs per visited (query, key) pair.
+Under torchrun every rank runs the same workload on its own GPU (independent
+replicas, weak scaling); the time is the max over ranks.
+
+The same JSON line also carries the decode workloads (tokens/s, cache GB/s)
+and the 128K prefill, each against its roofline, the oracle timed on the host
+cores as a baseline, and an end-to-end number through host buffers.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "HCA prefill TFLOP/s and decode tok/s (cache GB/s) vs B200 roofline"
+FLOP_PER_PAIR = 4 * 64 * 512
+BLOCK = 128
+WINDOW = 128
+
+
+# ---------------------------------------------------------------------------
+# work accounting (closed counts of the visibility rule; no attention math)
+# ---------------------------------------------------------------------------
+def nc_of(t: int) -> int:
+    return max(0, (t - WINDOW + 1) // BLOCK)
+
+
+def visited_pairs(T: int) -> int:
+    return sum(nc_of(t) + min(t + 1, WINDOW) for t in range(T))
+
+
+def prefill_bytes(B: int, T: int) -> int:
+    nb = T // BLOCK
+    return 2 * B * (3 * T * 64 * 512 + 2 * T * 512 + 2 * nb * 512 + T)
+
+
+def decode_cache_keys(lens):
+    return sum(min(max(0, (L - 128) // 128), 10 ** 9) + min(L, 128) for L in lens)
+
+
+# ---------------------------------------------------------------------------
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def read_traffic(kernel_file: str, summary: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the kernel source as it is now (sha256 of the file recorded beside it)."""
+    try:
+        vals = {}
+        with open(os.path.join(ROOT, "profiles", summary)) as f:
+            for line in f:
+                if "=" in line and not line.startswith("#"):
+                    a, b = line.strip().split("=", 1)
+                    vals[a.strip()] = b.strip()
+        src = open(os.path.join(ROOT, "compressed_sliding_window_b200", "csrc", kernel_file), "rb").read()
+        if hashlib.sha256(src).hexdigest() != vals.get("source_sha256"):
+            return None
+        return float(vals["traffic_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on a bounded sample of the same workload
+# ---------------------------------------------------------------------------
+def oracle_sample(cfg, positions):
+    """Time the oracle (compress + attention for `positions`); returns
+    (seconds, flops of the sampled rows)."""
+    import numpy as np
+    from compressed_sliding_window_b200 import inputs as I
+    from oracle import hca_oracle as O
+    chunks = sorted({p // I.CHUNK for p in positions})
+    x = I.prefill_inputs(cfg, chunks=chunks)
+    f64 = lambda t: t.float().numpy().astype(np.float64)  # noqa: E731
+    q = f64(x["q"][:, positions])
+    g = f64(x["g"][:, positions])
+    k, v, s = f64(x["k"]), f64(x["v"]), f64(x["s"])
+    t0 = time.perf_counter()
+    cache = O.compress(k, v, s)
+    O.prefill_forward(q, k, v, s, g, positions=positions, rows_only=True, cache=cache)
+    dt = time.perf_counter() - t0
+    pairs = sum(nc_of(t) + min(t + 1, WINDOW) for t in positions)
+    return dt, pairs * FLOP_PER_PAIR
+
+
+def cpu_baseline(cfg, n_pos=384):
+    T = cfg.T
+    positions = [int(round(i * (T - 1) / (n_pos - 1))) for i in range(n_pos)]
+    dt, fl = oracle_sample(cfg, positions)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": host_cores(), "kind": "oracle",
+            "sample": f"{n_pos} query positions evenly spaced over T={T} (all 64 heads), "
+                      f"plus the fp64 compression of all {T // BLOCK} blocks; {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------------------
+def setup_dist(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def flush_l2(buf):
+    buf.zero_()
+
+
+def run_ours(args):
+    import torch
+    import compressed_sliding_window_b200 as hca
+    from compressed_sliding_window_b200 import inputs as I
+
+    world, rank, local = setup_dist(args.gpus)
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    cfg = I.PREFILL_32K
+    B, T = cfg.B, cfg.T
+    pairs = visited_pairs(T)
+    flops = B * pairs * FLOP_PER_PAIR
+    x = I.prefill_inputs(cfg, pin=True)
+    d = {n: t.to(dev, non_blocking=True) for n, t in x.items()}
+    nb = T // BLOCK
+    ck = torch.empty((B, nb, 512), dtype=torch.bfloat16, device=dev)
+    cv = torch.empty_like(ck)
+    out = torch.empty_like(d["q"])
+    torch.cuda.synchronize()
+
+    def step():
+        hca.compress(d["k"], d["v"], d["s"], ck, cv)
+        hca.prefill(d["q"], d["k"], d["v"], ck, cv, d["g"], out=out)
+
+    for _ in range(args.warmup):
+        step()
+    barrier(world)
+    code, where = hca.device_error(dev)
+    if code != 0:
+        raise RuntimeError(f"device error {code} at {where} during warm-up")
+
+    stream = torch.cuda.current_stream(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                          else local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    t_start.record(stream)
+    for i in range(args.steps):
+        hca.compress(d["k"], d["v"], d["s"], ck, cv)
+        ev[i][0].record(stream)
+        hca.prefill(d["q"], d["k"], d["v"], ck, cv, d["g"], out=out)
+        ev[i][1].record(stream)
+    t_end.record(stream)
+    barrier(world)
+    clk = clocks.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    max_ms = max_over_ranks(elapsed_ms, world)
+    prefill_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    code, where = hca.device_error(dev)
+    if code != 0:
+        raise RuntimeError(f"device error {code} at {where} in the timed region")
+
+    value = world * flops * args.steps / (max_ms / 1e3) / 1e12
+    alg_bytes = prefill_bytes(B, T)
+    achieved_gbs = alg_bytes / (prefill_ms / 1e3) / 1e9
+    traffic = read_traffic("prefill.cuh", "prefill_T32768_traffic.txt")
+    result = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "HCA compress + prefill, B=1 T=32768 (K x0.5), 64 heads x 512, "
+                               "1 KV head, block 128, window 128",
+                   "global_batch": world * B, "seq_len": T, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (4.3 GB read per step)"},
+        "roofline": {"kernel": "prefill_kernel", "bound": "hbm", "achieved": achieved_gbs,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved_gbs / peaks["hbm_gbs"],
+                     "traffic": traffic, "peak_source": peaks["source"],
+                     "algorithmic_bytes": alg_bytes, "avg_launch_ms": prefill_ms,
+                     "tensor": {"achieved": flops / (prefill_ms / 1e3) / 1e12,
+                                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                "frac": flops / (prefill_ms / 1e3) / 1e12 / peaks["bf16_tflops"]}},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk,
+    }
+
+    # ---------------- end to end through host buffers (pinned) ----------------
+    hx = x
+    hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in hx.values())
+    d2h = hout.numel() * hout.element_size()
+
+    def e2e_step():
+        for n in d:
+            d[n].copy_(hx[n], non_blocking=True)
+        hca.compress(d["k"], d["v"], d["s"], ck, cv)
+        hca.prefill(d["q"], d["k"], d["v"], ck, cv, d["g"], out=out)
+        hout.copy_(out, non_blocking=True)
+
+    e2e_step()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    result["e2e"] = {"value": world * flops * args.e2e_steps / (e2e_ms / 1e3) / 1e12,
+                     "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                     "ms_per_step": e2e_ms / args.e2e_steps}
+    del d, out, hout, x, hx
+    torch.cuda.empty_cache()
+
+    if rank == 0 and not args.quick:
+        result["decode"] = [bench_decode(I.DECODE_64x128K, dev, peaks, args),
+                            bench_decode(I.DECODE_16xLONG, dev, peaks, args)]
+        result["prefill_128k"] = bench_prefill_128k(dev, peaks, args)
+    if rank == 0 and world == 1 and not args.no_cpu:
+        result["cpu_baseline"] = cpu_baseline(cfg)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def bench_prefill_128k(dev, peaks, args):
+    import torch
+    import compressed_sliding_window_b200 as hca
+    from compressed_sliding_window_b200 import inputs as I
+    cfg = I.PREFILL_128K
+    T = cfg.T
+    x = I.prefill_inputs(cfg)
+    d = {n: t.to(dev) for n, t in x.items()}
+    del x
+    nb = T // BLOCK
+    ck = torch.empty((1, nb, 512), dtype=torch.bfloat16, device=dev)
+    cv = torch.empty_like(ck)
+    out = torch.empty_like(d["q"])
+    for _ in range(3):
+        hca.compress(d["k"], d["v"], d["s"], ck, cv)
+        hca.prefill(d["q"], d["k"], d["v"], ck, cv, d["g"], out=out)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    n = args.steps_128k
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(n)]
+    for i in range(n):
+        hca.compress(d["k"], d["v"], d["s"], ck, cv)
+        ev[i][0].record(stream)
+        hca.prefill(d["q"], d["k"], d["v"], ck, cv, d["g"], out=out)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    code, where = hca.device_error(dev)
+    if code != 0:
+        raise RuntimeError(f"device error {code} at {where} (128K prefill)")
+    ms = sum(a.elapsed_time(b) for a, b in ev) / n
+    flops = visited_pairs(T) * FLOP_PER_PAIR
+    tf = flops / (ms / 1e3) / 1e12
+    res = {"workload": "HCA prefill B=1 T=131072, 1024 entries, gate fused",
+           "tflops": tf, "ms_per_launch": ms, "flops": flops,
+           "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"],
+                        "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"],
+                        "peak_source": peaks["source"]},
+           "hbm_gbs": prefill_bytes(1, T) / (ms / 1e3) / 1e9}
+    del d, out
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_decode(cfg, dev, peaks, args):
+    import torch
+    import compressed_sliding_window_b200 as hca
+    from compressed_sliding_window_b200 import inputs as I
+    lens = I.decode_ctx_lens(cfg)
+    S = cfg.S
+    if cfg.from_raw:
+        L = cfg.ctx
+        max_nc = L // BLOCK
+        ck = torch.empty((S, max_nc, 512), dtype=torch.bfloat16, device=dev)
+        cv = torch.empty_like(ck)
+        wk = torch.empty((S, 128, 512), dtype=torch.bfloat16, device=dev)
+        wv = torch.empty_like(wk)
+        for i in range(S):
+            k, v, s = I.decode_raw_sequence(cfg, i, L)
+            hca.compress(k[None].to(dev), v[None].to(dev), s[None].to(dev), ck[i:i + 1], cv[i:i + 1])
+            wk[i] = I.ring_window(k, L).to(dev)
+            wv[i] = I.ring_window(v, L).to(dev)
+    else:
+        max_nc = 8191
+        parts = [I.decode_direct_sequence(cfg, i, max_nc) for i in range(S)]
+        ck, cv, wk, wv = (torch.stack([p[j] for p in parts]).to(dev) for j in range(4))
+    q, g = I.decode_query(cfg)
+    q, g = q.to(dev), g.to(dev)
+    ctx = torch.tensor(lens, dtype=torch.int32, device=dev)
+    ws = torch.empty((hca.decode_workspace_size(S),), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(q)
+    flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        hca.decode(q, ck, cv, wk, wv, ctx, g, workspace=ws, out=out)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    times = []
+    for _ in range(args.decode_steps):
+        flush_l2(flush)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        hca.decode(q, ck, cv, wk, wv, ctx, g, workspace=ws, out=out)
+        b.record(stream)
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    code, where = hca.device_error(dev)
+    if code != 0:
+        raise RuntimeError(f"device error {code} at {where} (decode)")
+    ms = statistics.median(times)
+    keys = decode_cache_keys(lens)
+    cache_bytes = keys * 2 * 512 * 2
+    total_bytes = cache_bytes + 3 * S * 64 * 512 * 2
+    gbs = cache_bytes / (ms / 1e3) / 1e9
+    res = {"workload": cfg.name, "S": S, "ctx_len": lens if len(set(lens)) > 1 else lens[0],
+           "tok_per_s": S / (ms / 1e3), "ms_per_step": ms, "cache_gbs": gbs,
+           "total_gbs": total_bytes / (ms / 1e3) / 1e9,
+           "roofline": {"bound": "hbm", "achieved": total_bytes / (ms / 1e3) / 1e9,
+                        "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": total_bytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                        "peak_source": peaks["source"]},
+           "l2": "flushed (256 MB write) before every timed step", "gpu_launches_per_step": 3}
+    del ck, cv, wk, wv, flush, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from compressed_sliding_window_b200 import inputs as I
+    cfg = I.PREFILL_32K
+    T = cfg.T
+    per_step = args.ref_positions
+    total = 0.0
+    fl_total = 0
+    for i in range(args.warmup + args.steps):
+        positions = [int((j * 7919 + i * 104729) % T) for j in range(per_step)]
+        positions = sorted(set(positions))
+        dt, fl = oracle_sample(cfg, positions)
+        if i >= args.warmup:
+            total += dt
+            fl_total += fl
+    value = fl_total / total / 1e12
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "HCA compress + prefill, B=1 T=32768 (K x0.5), 64 heads x 512, "
+                               "1 KV head, block 128, window 128"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": host_cores(),
+                         "kind": "oracle",
+                         "sample": f"each step: fp64 compression of all blocks + {per_step} "
+                                   f"pseudo-random query positions (all heads)"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--quick", action="store_true", help="skip decode / 128K measurements")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--decode-steps", type=int, default=20)
+    ap.add_argument("--steps-128k", type=int, default=10)
+    ap.add_argument("--ref-positions", type=int, default=24)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,198 @@
+"""B200-native Heavily Compressed Attention (HCA) forward path.
+
+Python binding over the C ABI of ``libhca.so`` (declared in include/hca.h).
+The functions here only check and marshal arguments (device pointers, sizes,
+the current CUDA stream); every step of the computation runs in the library's
+CUDA kernels.  There is no fallback: if the library is missing or no CUDA
+device is present, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+from .build import LIB_PATH
+
+HEADS = 64
+HEAD_DIM = 512
+BLOCK = 128
+WINDOW = 128
+
+STATUS = {
+    0: "HCA_OK", 1: "HCA_ERR_INVALID_ARG", 2: "HCA_ERR_UNSUPPORTED", 3: "HCA_ERR_CUDA",
+    4: "HCA_ERR_TIMEOUT", 5: "HCA_ERR_DEVICE_INPUT",
+}
+
+
+class HCAError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {STATUS.get(code, code)}")
+        self.code = code
+
+
+_LIB = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libhca.so (built in-tree by ``build.py``)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m compressed_sliding_window_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.hca_compress.argtypes = [vp, vp, vp, i, i, vp, vp, vp]
+        L.hca_prefill_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, f, vp, vp, vp]
+        L.hca_decode_workspace_size.argtypes = [i]
+        L.hca_decode_workspace_size.restype = sz
+        L.hca_decode.argtypes = [vp, vp, vp, i, vp, vp, vp, vp, i, i, f, vp, sz, vp, vp]
+        L.hca_get_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
+        L.hca_selftest_bounded_wait.argtypes = [i, vp]
+        L.hca_status_string.argtypes = [i]
+        L.hca_status_string.restype = ctypes.c_char_p
+        L.hca_version.restype = i
+        for name in ("hca_compress", "hca_prefill_fwd", "hca_decode", "hca_get_device_error",
+                     "hca_selftest_bounded_wait"):
+            getattr(L, name).restype = i
+        _LIB = L
+    return _LIB
+
+
+def _stream(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check(t: torch.Tensor, name: str, shape=None, dtype=torch.bfloat16):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be on a CUDA device")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _ok(fn: str, code: int):
+    if code != 0:
+        raise HCAError(fn, code)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def compress(k: torch.Tensor, v: torch.Tensor, s: torch.Tensor,
+             ck: Optional[torch.Tensor] = None, cv: Optional[torch.Tensor] = None
+             ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Compressed cache entries for every complete 128-token block.
+
+    k, v: [B, T, 512] bf16; s: [B, T] bf16 -> (ck, cv) [B, T // 128, 512] bf16.
+    """
+    B, T, D = k.shape
+    _check(k, "k", (B, T, HEAD_DIM))
+    _check(v, "v", (B, T, HEAD_DIM))
+    _check(s, "s", (B, T))
+    nb = T // BLOCK
+    if ck is None:
+        ck = torch.empty((B, nb, HEAD_DIM), dtype=torch.bfloat16, device=k.device)
+    if cv is None:
+        cv = torch.empty((B, nb, HEAD_DIM), dtype=torch.bfloat16, device=k.device)
+    _check(ck, "ck", (B, nb, HEAD_DIM))
+    _check(cv, "cv", (B, nb, HEAD_DIM))
+    _ok("hca_compress", lib().hca_compress(k.data_ptr(), v.data_ptr(), s.data_ptr(), B, T,
+                                           _ptr(ck) if nb else None, _ptr(cv) if nb else None,
+                                           _stream(k.device)))
+    return ck, cv
+
+
+def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, ck: torch.Tensor,
+            cv: torch.Tensor, g: torch.Tensor, scale: Optional[float] = None,
+            out: Optional[torch.Tensor] = None, return_lse: bool = False):
+    """HCA prefill attention with the gate fused.
+
+    q, g: [B, T, 64, 512]; k, v: [B, T, 512]; ck, cv: [B, T // 128, 512]
+    -> out [B, T, 64, 512] bf16 (and lse [B, T, 64] fp32 when asked).
+    """
+    B, T, H, D = q.shape
+    _check(q, "q", (B, T, H, HEAD_DIM))
+    _check(g, "g", (B, T, H, HEAD_DIM))
+    _check(k, "k", (B, T, HEAD_DIM))
+    _check(v, "v", (B, T, HEAD_DIM))
+    nb = T // BLOCK
+    _check(ck, "ck", (B, nb, HEAD_DIM))
+    _check(cv, "cv", (B, nb, HEAD_DIM))
+    if scale is None:
+        scale = 1.0 / math.sqrt(HEAD_DIM)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(out, "out", (B, T, H, HEAD_DIM))
+    lse = torch.empty((B, T, H), dtype=torch.float32, device=q.device) if return_lse else None
+    _ok("hca_prefill_fwd", lib().hca_prefill_fwd(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(ck) if nb else None,
+        _ptr(cv) if nb else None, g.data_ptr(), B, T, H, ctypes.c_float(scale), out.data_ptr(),
+        _ptr(lse), _stream(q.device)))
+    return (out, lse) if return_lse else out
+
+
+def forward(q, k, v, s, g, scale: Optional[float] = None, return_lse: bool = False):
+    """Compress then prefill: the whole HCA forward for a prompt."""
+    ck, cv = compress(k, v, s)
+    return prefill(q, k, v, ck, cv, g, scale=scale, return_lse=return_lse)
+
+
+def decode_workspace_size(S: int) -> int:
+    return int(lib().hca_decode_workspace_size(S))
+
+
+def decode(q: torch.Tensor, ck: torch.Tensor, cv: torch.Tensor, wk: torch.Tensor,
+           wv: torch.Tensor, ctx_len: torch.Tensor, g: torch.Tensor,
+           scale: Optional[float] = None, workspace: Optional[torch.Tensor] = None,
+           out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One decode step: q, g [S, 64, 512]; ck, cv [S, max_nc, 512]; wk, wv
+    [S, 128, 512] ring windows; ctx_len [S] int32 on the device."""
+    S, H, D = q.shape
+    _check(q, "q", (S, H, HEAD_DIM))
+    _check(g, "g", (S, H, HEAD_DIM))
+    max_nc = ck.shape[1]
+    _check(ck, "ck", (S, max_nc, HEAD_DIM))
+    _check(cv, "cv", (S, max_nc, HEAD_DIM))
+    _check(wk, "wk", (S, WINDOW, HEAD_DIM))
+    _check(wv, "wv", (S, WINDOW, HEAD_DIM))
+    _check(ctx_len, "ctx_len", (S,), dtype=torch.int32)
+    if scale is None:
+        scale = 1.0 / math.sqrt(HEAD_DIM)
+    need = decode_workspace_size(S)
+    if workspace is None:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(out, "out", (S, H, HEAD_DIM))
+    _check(workspace, "workspace", dtype=torch.uint8)
+    _ok("hca_decode", lib().hca_decode(
+        q.data_ptr(), _ptr(ck) if max_nc else None, _ptr(cv) if max_nc else None, max_nc,
+        wk.data_ptr(), wv.data_ptr(), ctx_len.data_ptr(), g.data_ptr(), S, H,
+        ctypes.c_float(scale), workspace.data_ptr(), workspace.numel(), out.data_ptr(),
+        _stream(q.device)))
+    return out
+
+
+def device_error(device: Optional[torch.device] = None) -> Tuple[int, int]:
+    """(status, where) from the device-side error word (synchronises the stream)."""
+    device = device or torch.device("cuda", torch.cuda.current_device())
+    where = ctypes.c_uint(0)
+    code = lib().hca_get_device_error(_stream(device), ctypes.byref(where))
+    return code, where.value
+
+
+def selftest_bounded_wait(limit_us: int, device: Optional[torch.device] = None):
+    device = device or torch.device("cuda", torch.cuda.current_device())
+    _ok("hca_selftest_bounded_wait", lib().hca_selftest_bounded_wait(limit_us, _stream(device)))

@@ -1,0 +1,257 @@
+// libhca.so: the C ABI declared in include/hca.h.
+//
+// Host-side work only: argument validation, TMA tensor-map encoding, grid
+// sizing and launches.  Every step of the computation runs in the kernels
+// included below.  One translation unit, so the device-side error word is a
+// single symbol shared by all kernels.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/hca.h"
+#include "hca_ptx.cuh"
+#include "compress.cuh"
+#include "prefill.cuh"
+#include "decode.cuh"
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 3-D bf16 tensor [Z][Y][X] (X contiguous, X = 512), box (64, box_y, 1),
+// 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* m, const void* base, uint64_t X, uint64_t Y, uint64_t Z,
+              uint32_t box_y) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[3] = {X, Y, Z};
+  const cuuint64_t strides[2] = {X * 2, X * Y * 2};
+  const cuuint32_t box[3] = {64, box_y, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+hca_status_t launch_status() {
+  return cudaGetLastError() == cudaSuccess ? HCA_OK : HCA_ERR_CUDA;
+}
+
+int device_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  return sms;
+}
+
+bool scale_ok(float scale) { return std::isfinite(scale) && scale > 0.f; }
+
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar_storage;
+  __shared__ int abort_flag;
+  const uint32_t b = hca::smem_u32(&bar_storage);
+  if (threadIdx.x == 0) {
+    hca::mbar_init(b, 1);
+    abort_flag = 0;
+    hca::fence_mbar_init();
+  }
+  __syncthreads();
+  // Nobody arrives: the wait must give up after limit_ns and record a timeout.
+  hca::mbar_wait(b, 0, &abort_flag, limit_ns, 900);
+}
+
+}  // namespace
+
+extern "C" {
+
+hca_status_t hca_compress(const hca_bf16* k, const hca_bf16* v, const hca_bf16* s, int B, int T,
+                          hca_bf16* ck, hca_bf16* cv, hca_stream_t stream) {
+  if (B < 1 || T < 1 || k == nullptr || v == nullptr || s == nullptr) return HCA_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v)) return HCA_ERR_INVALID_ARG;
+  const int nb = T / HCA_BLOCK;
+  if (nb == 0) return HCA_OK;
+  if (ck == nullptr || cv == nullptr) return HCA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * nb > 0x7fffffffLL) return HCA_ERR_UNSUPPORTED;
+  dim3 grid(B * nb, 8);
+  hca::compress_kernel<<<grid, hca::kCompressThreads, 0, stream>>>(k, v, s, T, nb, ck, cv);
+  return launch_status();
+}
+
+hca_status_t hca_prefill_fwd(const hca_bf16* q, const hca_bf16* k, const hca_bf16* v,
+                             const hca_bf16* ck, const hca_bf16* cv, const hca_bf16* g, int B,
+                             int T, int H, float scale, hca_bf16* out, float* lse,
+                             hca_stream_t stream) {
+  namespace P = hca::prefill;
+  if (H != HCA_NUM_HEADS) return HCA_ERR_UNSUPPORTED;
+  if (B < 1 || T < 1 || !scale_ok(scale)) return HCA_ERR_INVALID_ARG;
+  if (q == nullptr || k == nullptr || v == nullptr || g == nullptr || out == nullptr)
+    return HCA_ERR_INVALID_ARG;
+  const int nb = T / HCA_BLOCK;
+  if (nb > 0 && (ck == nullptr || cv == nullptr)) return HCA_ERR_INVALID_ARG;
+  const void* ptrs[7] = {q, k, v, g, out, ck, cv};
+  for (const void* ptr : ptrs)
+    if (ptr != nullptr && !aligned16(ptr)) return HCA_ERR_INVALID_ARG;
+  if (static_cast<long long>(T) * HCA_NUM_HEADS > 0x7fffffffLL) return HCA_ERR_UNSUPPORTED;
+  const long long row_tiles = (T + 1) / 2;
+  const long long items = static_cast<long long>(B) * row_tiles * 2;
+  if (items > 0x7fffffffLL) return HCA_ERR_UNSUPPORTED;
+
+  P::Maps maps;
+  const uint64_t rows = static_cast<uint64_t>(T) * HCA_NUM_HEADS;
+  bool ok = make_map(&maps.q, q, HCA_HEAD_DIM, rows, B, 128) &&
+            make_map(&maps.g, g, HCA_HEAD_DIM, rows, B, 128) &&
+            make_map(&maps.out, out, HCA_HEAD_DIM, rows, B, 128) &&
+            make_map(&maps.k, k, HCA_HEAD_DIM, T, B, 128) &&
+            make_map(&maps.v, v, HCA_HEAD_DIM, T, B, 128) &&
+            make_map(&maps.k16, k, HCA_HEAD_DIM, T, B, 16) &&
+            make_map(&maps.v16, v, HCA_HEAD_DIM, T, B, 16);
+  if (ok && nb > 0) {
+    ok = make_map(&maps.ck, ck, HCA_HEAD_DIM, nb, B, 128) &&
+         make_map(&maps.cv, cv, HCA_HEAD_DIM, nb, B, 128);
+  } else if (ok) {  // no compressed entry exists; the maps are never used
+    maps.ck = maps.k;
+    maps.cv = maps.v;
+  }
+  if (!ok) return HCA_ERR_CUDA;
+
+  P::Params prm;
+  prm.B = B;
+  prm.T = T;
+  prm.row_tiles = static_cast<int>(row_tiles);
+  prm.items = static_cast<int>(items);
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.lse = lse;
+  const int sms = device_sms();
+  if (sms <= 0) return HCA_ERR_CUDA;
+  const int grid = static_cast<int>(items < sms ? items : sms);
+  if (cudaFuncSetAttribute(P::prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           P::kSmemAlloc) != cudaSuccess)
+    return HCA_ERR_CUDA;
+  P::prefill_kernel<<<grid, P::kThreads, P::kSmemAlloc, stream>>>(maps, prm);
+  return launch_status();
+}
+
+size_t hca_decode_workspace_size(int S) {
+  if (S < 1) return 0;
+  const int sms = device_sms();
+  if (sms <= 0) return 0;
+  const int slots = sms + S;
+  // partial O and (m, l) per slot, then the tile prefix [S + 1] int64
+  return hca::decode::ws_bytes(slots) + 256 + static_cast<size_t>(S + 1) * 8;
+}
+
+hca_status_t hca_decode(const hca_bf16* q, const hca_bf16* ck, const hca_bf16* cv, int max_nc,
+                        const hca_bf16* wk, const hca_bf16* wv, const int32_t* ctx_len,
+                        const hca_bf16* g, int S, int H, float scale, void* ws, size_t ws_bytes,
+                        hca_bf16* out, hca_stream_t stream) {
+  namespace D = hca::decode;
+  if (H != HCA_NUM_HEADS) return HCA_ERR_UNSUPPORTED;
+  if (S < 1 || max_nc < 0 || !scale_ok(scale)) return HCA_ERR_INVALID_ARG;
+  if (q == nullptr || wk == nullptr || wv == nullptr || ctx_len == nullptr || g == nullptr ||
+      out == nullptr || ws == nullptr)
+    return HCA_ERR_INVALID_ARG;
+  if (max_nc > 0 && (ck == nullptr || cv == nullptr)) return HCA_ERR_INVALID_ARG;
+  const void* ptrs[7] = {q, wk, wv, g, out, ck, cv};
+  for (const void* ptr : ptrs)
+    if (ptr != nullptr && !aligned16(ptr)) return HCA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return HCA_ERR_INVALID_ARG;
+  if (ws_bytes < hca_decode_workspace_size(S)) return HCA_ERR_INVALID_ARG;
+  if (static_cast<long long>(S) * HCA_NUM_HEADS > 0x7fffffffLL || S > 65535)
+    return HCA_ERR_UNSUPPORTED;
+
+  const int sms = device_sms();
+  if (sms <= 0) return HCA_ERR_CUDA;
+  const int slots = sms + S;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  D::Params prm;
+  prm.ctx_len = ctx_len;
+  prm.S = S;
+  prm.max_nc = max_nc;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.ws_o = reinterpret_cast<float*>(wsb);
+  prm.ws_ml = reinterpret_cast<float*>(wsb + D::ws_o_bytes(slots));
+  prm.seq_tile = reinterpret_cast<long long*>(wsb + ((D::ws_bytes(slots) + 255) & ~size_t(255)));
+
+  D::Maps maps;
+  bool ok = make_map(&maps.q, q, HCA_HEAD_DIM, static_cast<uint64_t>(S) * HCA_NUM_HEADS, 1, 64) &&
+            make_map(&maps.wk, wk, HCA_HEAD_DIM, HCA_WINDOW, S, 128) &&
+            make_map(&maps.wv, wv, HCA_HEAD_DIM, HCA_WINDOW, S, 128);
+  if (ok && max_nc > 0) {
+    ok = make_map(&maps.ck, ck, HCA_HEAD_DIM, max_nc, S, 128) &&
+         make_map(&maps.cv, cv, HCA_HEAD_DIM, max_nc, S, 128);
+  } else if (ok) {
+    maps.ck = maps.wk;
+    maps.cv = maps.wv;
+  }
+  if (!ok) return HCA_ERR_CUDA;
+
+  D::plan_kernel<<<1, 1024, 0, stream>>>(ctx_len, S, max_nc, prm.seq_tile);
+  if (cudaGetLastError() != cudaSuccess) return HCA_ERR_CUDA;
+  if (cudaFuncSetAttribute(D::decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           D::kSmemAlloc) != cudaSuccess)
+    return HCA_ERR_CUDA;
+  D::decode_kernel<<<sms, D::kThreads, D::kSmemAlloc, stream>>>(maps, prm);
+  if (cudaGetLastError() != cudaSuccess) return HCA_ERR_CUDA;
+  D::combine_kernel<<<dim3(S, HCA_NUM_HEADS), 128, 0, stream>>>(prm, sms, g, out);
+  return launch_status();
+}
+
+hca_status_t hca_get_device_error(hca_stream_t stream, unsigned int* where) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return HCA_ERR_CUDA;
+  unsigned int word = 0, w = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&word, hca::g_error_word, sizeof(word)) != cudaSuccess)
+    return HCA_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&w, hca::g_error_where, sizeof(w)) != cudaSuccess) return HCA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(hca::g_error_word, &zero, sizeof(zero)) != cudaSuccess ||
+      cudaMemcpyToSymbol(hca::g_error_where, &zero, sizeof(zero)) != cudaSuccess)
+    return HCA_ERR_CUDA;
+  if (where != nullptr) *where = w;
+  if (word & hca::DEVERR_TIMEOUT) return HCA_ERR_TIMEOUT;
+  if (word & hca::DEVERR_BAD_INPUT) return HCA_ERR_DEVICE_INPUT;
+  return HCA_OK;
+}
+
+hca_status_t hca_selftest_bounded_wait(int limit_us, hca_stream_t stream) {
+  if (limit_us < 1 || limit_us > 10000000) return HCA_ERR_INVALID_ARG;
+  selftest_wait_kernel<<<1, 32, 0, stream>>>(static_cast<uint64_t>(limit_us) * 1000ull);
+  return launch_status();
+}
+
+const char* hca_status_string(hca_status_t status) {
+  switch (status) {
+    case HCA_OK: return "HCA_OK";
+    case HCA_ERR_INVALID_ARG: return "HCA_ERR_INVALID_ARG";
+    case HCA_ERR_UNSUPPORTED: return "HCA_ERR_UNSUPPORTED";
+    case HCA_ERR_CUDA: return "HCA_ERR_CUDA";
+    case HCA_ERR_TIMEOUT: return "HCA_ERR_TIMEOUT";
+    case HCA_ERR_DEVICE_INPUT: return "HCA_ERR_DEVICE_INPUT";
+  }
+  return "HCA_ERR_UNKNOWN";
+}
+
+int hca_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,151 @@
+/*
+ * hca.h — C ABI of libhca.so, a B200 (sm_100a) implementation of the forward
+ * hot path of Heavily Compressed Attention (HCA).
+ *
+ * The method.  'BaiduがERNIE 5.5 Flash Baseを公開' §2.1 (Latent-Gated Sparse
+ * Attention) and its Chinese twin 'ERNIE 5.5 Flash Base 正式发布' §2.1 describe
+ * HCA layers that turn every 128 tokens into one cache entry and run one dense
+ * softmax over all of those entries plus a short window of recent raw tokens,
+ * with 64 query heads of width 512; every layer multiplies its attention
+ * output by a learned gate.  The xenospectrum analysis of the same release
+ * (section 活性140億パラメータと長文処理を支える仕組み) gives the window: the
+ * newest 128 tokens, kept uncompressed.  Where the pages are silent this
+ * library fixes: one shared KV head; entry j = softmax(s over block j)-weighted
+ * sum of the block's K rows (and, with the same weights, of its V rows), with s
+ * a per-token score; query t sees entry j only when block j lies wholly before
+ * its window, i.e. j < nc(t) = max(0, floor((t - 127) / 128)), and the raw keys
+ * max(0, t - 127) .. t; out = sigmoid(g) * o elementwise.
+ *
+ * Conventions shared by every call:
+ *  - bf16 values are passed as raw 16-bit patterns (hca_bf16).  Every tensor is
+ *    dense, row-major, on the current CUDA device, and 16-byte aligned.
+ *  - The caller owns every buffer and the stream; the library allocates no
+ *    memory and keeps no per-call state.  Calls are asynchronous on `stream`
+ *    (NULL = legacy default stream).
+ *  - Arguments are validated on the host before anything is launched; a
+ *    rejected call returns HCA_ERR_INVALID_ARG or HCA_ERR_UNSUPPORTED and
+ *    launches nothing.  HCA_ERR_CUDA reports a launch failure.
+ *  - Kernels never trap.  Every wait inside them is bounded; a wait that runs
+ *    out, or a device-resident argument found out of range (decode context
+ *    lengths), is recorded in a device-side error word that
+ *    hca_get_device_error() reads back.
+ *  - No C++ exception crosses this interface.
+ */
+#ifndef HCA_H
+#define HCA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HCA_OK = 0,
+  HCA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or scale       */
+  HCA_ERR_UNSUPPORTED = 2, /* a shape outside what the kernels implement       */
+  HCA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed                */
+  HCA_ERR_TIMEOUT = 4,     /* a device-side bounded wait ran out               */
+  HCA_ERR_DEVICE_INPUT = 5 /* a device-resident argument was out of range      */
+} hca_status_t;
+
+typedef uint16_t hca_bf16;              /* raw bfloat16 bits                   */
+typedef struct CUstream_st* hca_stream_t; /* same type as cudaStream_t         */
+
+#define HCA_HEAD_DIM 512 /* width of q, k, v and o rows                        */
+#define HCA_NUM_HEADS 64 /* query heads sharing the single KV head             */
+#define HCA_BLOCK 128    /* tokens per compressed entry                        */
+#define HCA_WINDOW 128   /* raw tokens each query attends (itself included)    */
+
+/*
+ * hca_compress — block compressor.
+ *   'BaiduがERNIE 5.5 Flash Baseを公開' §2.1: 128 tokens -> one cache entry.
+ *   For every complete block j < nb = floor(T / 128) of every batch b:
+ *     w = softmax(s[b, 128j : 128j + 128])            (fp32)
+ *     ck[b, j, :] = sum_i w_i * k[b, 128j + i, :]      (fp32 accumulate, bf16 RNE)
+ *     cv[b, j, :] = sum_i w_i * v[b, 128j + i, :]
+ *   Tokens of a trailing partial block are not compressed.
+ * Layout:  k, v  [B, T, 512] bf16;  s [B, T] bf16;  ck, cv [B, nb, 512] bf16.
+ * Errors:  B < 1 or T < 1 -> HCA_ERR_INVALID_ARG.  nb == 0 launches nothing.
+ */
+hca_status_t hca_compress(const hca_bf16* k, const hca_bf16* v, const hca_bf16* s, int B, int T,
+                          hca_bf16* ck, hca_bf16* cv, hca_stream_t stream);
+
+/*
+ * hca_prefill_fwd — HCA attention for every position of B sequences.
+ *   For query t of batch b and head h (page sources as above):
+ *     keys   = [ck[b, 0 : nc(t)] ; k[b, max(0, t-127) : t+1]]
+ *     values = [cv[b, 0 : nc(t)] ; v[b, max(0, t-127) : t+1]]
+ *     p      = softmax(scale * keys . q[b, t, h])      (one softmax over both sets)
+ *     out[b, t, h, :] = sigmoid(g[b, t, h, :]) * (p . values)
+ *   lse (optional) receives ln(sum exp(scale * keys . q)) per (b, t, h).
+ * Layout:  q, g, out [B, T, H, 512] bf16 (H = 64);  k, v [B, T, 512] bf16;
+ *          ck, cv [B, floor(T/128), 512] bf16 as written by hca_compress;
+ *          lse [B, T, H] fp32 or NULL.
+ * Errors:  H != 64 -> HCA_ERR_UNSUPPORTED; B < 1, T < 1, a null pointer (other
+ *          than lse), a pointer not 16-byte aligned, or a non-finite or
+ *          non-positive scale -> HCA_ERR_INVALID_ARG.
+ */
+hca_status_t hca_prefill_fwd(const hca_bf16* q, const hca_bf16* k, const hca_bf16* v,
+                             const hca_bf16* ck, const hca_bf16* cv, const hca_bf16* g, int B,
+                             int T, int H, float scale, hca_bf16* out, float* lse,
+                             hca_stream_t stream);
+
+/*
+ * hca_decode_workspace_size — bytes of scratch hca_decode needs for S
+ * sequences on the current device (partial results of the split-KV pass).
+ */
+size_t hca_decode_workspace_size(int S);
+
+/*
+ * hca_decode — one new token per sequence (split-KV over all SMs, then a
+ * log-sum-exp combine).
+ *   For sequence i with context length L = ctx_len[i] (which counts the new
+ *   token, so the query sits at t = L - 1):
+ *     keys   = [ck[i, 0 : nc(L-1)] ; the min(L, 128) newest raw keys]
+ *     out[i, h, :] = sigmoid(g[i, h, :]) * softmax(scale * keys . q[i, h]) . values
+ *   The raw window is a ring: the token at position p lives in slot p mod 128
+ *   of wk/wv; when L < 128 only slots 0 .. L-1 are read.  Slot order does not
+ *   change the result (no positional term).
+ * Layout:  q, g, out [S, H, 512] bf16 (H = 64);  ck, cv [S, max_nc, 512] bf16;
+ *          wk, wv [S, 128, 512] bf16;  ctx_len [S] int32 on the device;
+ *          ws: caller-owned device scratch of at least
+ *          hca_decode_workspace_size(S) bytes, 256-byte aligned.
+ * Errors:  host-checked as for prefill (and ws_bytes too small ->
+ *          HCA_ERR_INVALID_ARG).  A device-side ctx_len < 1 or one needing more
+ *          than max_nc entries is clamped and reported later by
+ *          hca_get_device_error() as HCA_ERR_DEVICE_INPUT.
+ */
+hca_status_t hca_decode(const hca_bf16* q, const hca_bf16* ck, const hca_bf16* cv, int max_nc,
+                        const hca_bf16* wk, const hca_bf16* wv, const int32_t* ctx_len,
+                        const hca_bf16* g, int S, int H, float scale, void* ws, size_t ws_bytes,
+                        hca_bf16* out, hca_stream_t stream);
+
+/*
+ * hca_get_device_error — synchronises `stream`, then reads and clears the
+ * device-side error word of the current device.  Returns HCA_OK,
+ * HCA_ERR_TIMEOUT, HCA_ERR_DEVICE_INPUT or HCA_ERR_CUDA.  `where`, if not
+ * NULL, receives an internal code naming the wait that gave up.
+ */
+hca_status_t hca_get_device_error(hca_stream_t stream, unsigned int* where);
+
+/*
+ * hca_selftest_bounded_wait — launches one CTA that waits on an mbarrier
+ * nobody arrives on, with a limit of `limit_us` microseconds (1 .. 10^7).
+ * The kernel gives up, records HCA_ERR_TIMEOUT and exits normally; the
+ * context stays usable.  Exists to test the failure path without faulting.
+ */
+hca_status_t hca_selftest_bounded_wait(int limit_us, hca_stream_t stream);
+
+/* hca_status_string — static, human-readable name of a status code. */
+const char* hca_status_string(hca_status_t status);
+
+/* hca_version — library version as major*10000 + minor*100 + patch. */
+int hca_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HCA_H */

@@ -143,9 +143,10 @@ def attend(qrows: np.ndarray, keys: np.ndarray, values: np.ndarray,
     return o, lse
 
 
-def _prefill_rows(qb, gb, kb, vb, ckb, cvb, positions: np.ndarray,
+def _prefill_rows(qrows, grows, kb, vb, ckb, cvb, positions: np.ndarray,
                   blk: int, win: int, scale: float):
-    """Outputs for the given query positions of one sequence.
+    """Outputs for the given query positions of one sequence; qrows, grows
+    [len(positions), H, D] are the query and gate rows of those positions.
 
     The key set is the union over these positions: the compressed entries
     0 .. max nc - 1 and the raw tokens from the earliest window start to the
@@ -163,8 +164,8 @@ def _prefill_rows(qb, gb, kb, vb, ckb, cvb, positions: np.ndarray,
         t = int(t)
         mask[row, :n_c] = ent_idx < num_visible_blocks(t, blk, win)
         mask[row, n_c:] = (raw_idx >= window_start(t, win)) & (raw_idx <= t)
-    o, lse = attend(qb[positions], keys, vals, mask, scale)
-    out = sigmoid(gb[positions]) * o
+    o, lse = attend(qrows, keys, vals, mask, scale)
+    out = sigmoid(grows) * o
     return out, lse
 
 
@@ -172,19 +173,19 @@ def prefill_forward(q, k, v, s, g, blk: int = BLOCK, win: int = WINDOW,
                     scale: Optional[float] = None,
                     positions: Optional[Sequence[int]] = None,
                     round_cache_bf16: bool = False, chunk: int = 128,
-                    return_lse: bool = False, cache=None):
+                    return_lse: bool = False, cache=None, rows_only: bool = False):
     """HCA prefill forward in fp64.
 
     q, g: [B, T, H, D]; k, v: [B, T, D]; s: [B, T].  Returns out [B, T, H, D]
     (or [B, len(positions), H, D] when `positions` selects rows), and the lse
-    [.., H] when asked.  `cache` may pass precomputed (cK, cV) from
-    ``compress`` to avoid recomputing them.
+    [.., H] when asked.  With ``rows_only`` q and g hold just the selected rows
+    ([B, len(positions), H, D], in the order of `positions`).  `cache` may pass
+    precomputed (cK, cV) from ``compress``.
     """
-    q = np.asarray(q, dtype=np.float64)
-    g = np.asarray(g, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
-    B, T, H, D = q.shape
+    B, T, D = k.shape
+    H = q.shape[2]
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     ck, cv = cache if cache is not None else compress(k, v, s, blk)
@@ -193,12 +194,24 @@ def prefill_forward(q, k, v, s, g, blk: int = BLOCK, win: int = WINDOW,
     pos = np.arange(T) if positions is None else np.asarray(list(positions), dtype=np.int64)
     out = np.empty((B, len(pos), H, D), dtype=np.float64)
     lse = np.empty((B, len(pos), H), dtype=np.float64)
+    # group the requested rows so that every group lies inside one `chunk`-long
+    # stretch of positions (keeps each group's key set short)
+    order = np.argsort(pos, kind="stable")
+    groups = []
+    start = 0
+    for n in range(1, len(order) + 1):
+        if n == len(order) or pos[order[n]] // chunk != pos[order[start]] // chunk:
+            groups.append(order[start:n])
+            start = n
     for b in range(B):
-        for c0 in range(0, len(pos), chunk):
-            sel = pos[c0 : c0 + chunk]
-            o, l = _prefill_rows(q[b], g[b], k[b], v[b], ck[b], cv[b], sel, blk, win, scale)
-            out[b, c0 : c0 + chunk] = o
-            lse[b, c0 : c0 + chunk] = l
+        for idx in groups:
+            sel = pos[idx]
+            rows = idx if rows_only else sel
+            qr = np.asarray(q[b][rows], dtype=np.float64)
+            gr = np.asarray(g[b][rows], dtype=np.float64)
+            o, l = _prefill_rows(qr, gr, k[b], v[b], ck[b], cv[b], sel, blk, win, scale)
+            out[b, idx] = o
+            lse[b, idx] = l
     return (out, lse) if return_lse else out
 
 

@@ -1,0 +1,113 @@
+"""Host-only checks of the C ABI: the library builds and loads without a GPU,
+exports every function include/hca.h declares, and rejects bad arguments
+before launching anything (these calls never reach a kernel)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from compressed_sliding_window_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    path = B.build()
+    return ctypes.CDLL(path)
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "hca.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(hca_[a-z0-9_]+)\s*\(", text)
+    assert names, "no declarations found"
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_expected_entry_points_declared():
+    names = set(declared_functions())
+    for n in ("hca_compress", "hca_prefill_fwd", "hca_decode", "hca_decode_workspace_size",
+              "hca_get_device_error", "hca_status_string", "hca_version"):
+        assert n in names
+
+
+def test_status_strings(lib):
+    lib.hca_status_string.restype = ctypes.c_char_p
+    assert lib.hca_status_string(0) == b"HCA_OK"
+    assert lib.hca_status_string(1) == b"HCA_ERR_INVALID_ARG"
+    assert lib.hca_status_string(4) == b"HCA_ERR_TIMEOUT"
+    assert lib.hca_status_string(99) == b"HCA_ERR_UNKNOWN"
+    assert lib.hca_version() >= 100
+
+
+def test_compress_rejects_bad_args(lib):
+    lib.hca_compress.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 2 + [ctypes.c_void_p] * 3
+    fake = 0x10000
+    assert lib.hca_compress(None, fake, fake, 1, 256, fake, fake, None) == 1
+    assert lib.hca_compress(fake, fake, fake, 0, 256, fake, fake, None) == 1
+    assert lib.hca_compress(fake, fake, fake, 1, 0, fake, fake, None) == 1
+    assert lib.hca_compress(fake + 2, fake, fake, 1, 256, fake, fake, None) == 1   # misaligned
+    assert lib.hca_compress(fake, fake, fake, 1, 256, None, fake, None) == 1      # no output
+    assert lib.hca_compress(fake, fake, fake, 1, 100, None, None, None) == 0      # nb = 0: no-op
+
+
+def test_prefill_rejects_bad_args(lib):
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    lib.hca_prefill_fwd.argtypes = [vp] * 6 + [i, i, i, ctypes.c_float, vp, vp, vp]
+    f = 0x10000
+    ok_args = [f, f, f, f, f, f, 1, 256, 64, 0.04, f, None, None]
+
+    def call(**kw):
+        a = list(ok_args)
+        names = ["q", "k", "v", "ck", "cv", "g", "B", "T", "H", "scale", "out", "lse", "st"]
+        for k2, v2 in kw.items():
+            a[names.index(k2)] = v2
+        return lib.hca_prefill_fwd(*a)
+
+    assert call(H=63) == 2
+    assert call(B=0) == 1
+    assert call(T=0) == 1
+    assert call(scale=float("nan")) == 1
+    assert call(scale=-1.0) == 1
+    assert call(q=None) == 1
+    assert call(out=None) == 1
+    assert call(ck=None) == 1          # T = 256 has compressed entries
+    assert call(g=f + 8) == 1          # misaligned
+
+
+def test_decode_rejects_bad_args(lib):
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    lib.hca_decode.argtypes = [vp, vp, vp, i, vp, vp, vp, vp, i, i, ctypes.c_float, vp,
+                               ctypes.c_size_t, vp, vp]
+    f = 0x10000
+    assert lib.hca_decode(f, f, f, 8, f, f, f, f, 4, 32, 0.04, f, 1 << 30, f, None) == 2
+    assert lib.hca_decode(f, f, f, 8, f, f, f, f, 0, 64, 0.04, f, 1 << 30, f, None) == 1
+    assert lib.hca_decode(None, f, f, 8, f, f, f, f, 4, 64, 0.04, f, 1 << 30, f, None) == 1
+    assert lib.hca_decode(f, f, f, 8, f, f, None, f, 4, 64, 0.04, f, 1 << 30, f, None) == 1
+    assert lib.hca_decode(f, f, f, -1, f, f, f, f, 4, 64, 0.04, f, 1 << 30, f, None) == 1
+    assert lib.hca_decode(f, f, f, 8, f, f, f, f, 4, 64, 0.0, f, 1 << 30, f, None) == 1
+    assert lib.hca_decode(f, f, f, 8, f, f, f, f, 4, 64, 0.04, f + 16, 1 << 30, f, None) == 1
+
+
+def test_selftest_rejects_bad_limit(lib):
+    lib.hca_selftest_bounded_wait.argtypes = [ctypes.c_int, ctypes.c_void_p]
+    assert lib.hca_selftest_bounded_wait(0, None) == 1
+    assert lib.hca_selftest_bounded_wait(10 ** 8, None) == 1
+
+
+def test_python_binding_fails_loudly_without_gpu():
+    import torch
+    import compressed_sliding_window_b200 as hca
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    x = torch.zeros((1, 256, 512), dtype=torch.bfloat16)
+    s = torch.zeros((1, 256), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        hca.compress(x, x, s)
