@@ -219,6 +219,103 @@ hca_status_t hca_decode(const hca_bf16* q, const hca_bf16* ck, const hca_bf16* c
   return launch_status();
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// No-allocation decode: the same kernels as hca_decode, with their scratch in
+// a fixed device array owned by the library.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int kNoAllocSlots = HCA_NOALLOC_MAX_CTAS + HCA_NOALLOC_MAX_SEQS;
+// per slot: partial O [64][512] fp32 + (m, l) [2][64] fp32
+constexpr size_t kNoAllocSlotBytes = static_cast<size_t>(64) * 512 * 4 + 2 * 64 * 4;
+constexpr size_t kNoAllocPrefixOffset =
+    (kNoAllocSlots * kNoAllocSlotBytes + 255) & ~static_cast<size_t>(255);
+constexpr size_t kNoAllocScratchBytes =
+    kNoAllocPrefixOffset + static_cast<size_t>(HCA_NOALLOC_MAX_SEQS + 1) * 8;
+
+// Partial O / (m, l) of up to kNoAllocSlots split slots, then the tile prefix.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device (looked up once
+// per device, with that device current).  Null on failure.
+void* noalloc_scratch_address() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_addr[dev] = ptr;
+  }
+  return g_noalloc_addr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+hca_status_t hca_decode_noalloc(const hca_bf16* q, const hca_bf16* ck, const hca_bf16* cv,
+                                int max_nc, const hca_bf16* wk, const hca_bf16* wv,
+                                const int32_t* ctx_len, const hca_bf16* g, int S, int H,
+                                float scale, hca_bf16* out, hca_stream_t stream) {
+  namespace D = hca::decode;
+  if (H != HCA_NUM_HEADS) return HCA_ERR_UNSUPPORTED;
+  if (S < 1 || max_nc < 0 || !scale_ok(scale)) return HCA_ERR_INVALID_ARG;
+  if (S > HCA_NOALLOC_MAX_SEQS) return HCA_ERR_UNSUPPORTED;
+  if (q == nullptr || wk == nullptr || wv == nullptr || ctx_len == nullptr || g == nullptr ||
+      out == nullptr)
+    return HCA_ERR_INVALID_ARG;
+  if (max_nc > 0 && (ck == nullptr || cv == nullptr)) return HCA_ERR_INVALID_ARG;
+  const void* ptrs[7] = {q, wk, wv, g, out, ck, cv};
+  for (const void* ptr : ptrs)
+    if (ptr != nullptr && !aligned16(ptr)) return HCA_ERR_INVALID_ARG;
+
+  const int sms = device_sms();
+  if (sms <= 0) return HCA_ERR_CUDA;
+  const int grid = sms < HCA_NOALLOC_MAX_CTAS ? sms : HCA_NOALLOC_MAX_CTAS;
+  const int slots = grid + S;
+  uint8_t* wsb = static_cast<uint8_t*>(noalloc_scratch_address());
+  if (wsb == nullptr) return HCA_ERR_CUDA;
+
+  D::Params prm;
+  prm.ctx_len = ctx_len;
+  prm.S = S;
+  prm.max_nc = max_nc;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.ws_o = reinterpret_cast<float*>(wsb);
+  prm.ws_ml = reinterpret_cast<float*>(wsb + D::ws_o_bytes(slots));
+  prm.seq_tile = reinterpret_cast<long long*>(wsb + kNoAllocPrefixOffset);
+
+  D::Maps maps;
+  bool ok = make_map(&maps.q, q, HCA_HEAD_DIM, static_cast<uint64_t>(S) * HCA_NUM_HEADS, 1, 64) &&
+            make_map(&maps.wk, wk, HCA_HEAD_DIM, HCA_WINDOW, S, 128) &&
+            make_map(&maps.wv, wv, HCA_HEAD_DIM, HCA_WINDOW, S, 128);
+  if (ok && max_nc > 0) {
+    ok = make_map(&maps.ck, ck, HCA_HEAD_DIM, max_nc, S, 128) &&
+         make_map(&maps.cv, cv, HCA_HEAD_DIM, max_nc, S, 128);
+  } else if (ok) {
+    maps.ck = maps.wk;
+    maps.cv = maps.wv;
+  }
+  if (!ok) return HCA_ERR_CUDA;
+
+  D::plan_kernel<<<1, 1024, 0, stream>>>(ctx_len, S, max_nc, prm.seq_tile);
+  if (cudaGetLastError() != cudaSuccess) return HCA_ERR_CUDA;
+  if (cudaFuncSetAttribute(D::decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           D::kSmemAlloc) != cudaSuccess)
+    return HCA_ERR_CUDA;
+  D::decode_kernel<<<grid, D::kThreads, D::kSmemAlloc, stream>>>(maps, prm);
+  if (cudaGetLastError() != cudaSuccess) return HCA_ERR_CUDA;
+  D::combine_kernel<<<dim3(S, HCA_NUM_HEADS), 128, 0, stream>>>(prm, grid, g, out);
+  return launch_status();
+}
+
 hca_status_t hca_get_device_error(hca_stream_t stream, unsigned int* where) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return HCA_ERR_CUDA;
   unsigned int word = 0, w = 0, zero = 0;

@@ -123,6 +123,35 @@ hca_status_t hca_decode(const hca_bf16* q, const hca_bf16* ck, const hca_bf16* c
                         hca_bf16* out, hca_stream_t stream);
 
 /*
+ * hca_decode_noalloc — hca_decode for callers that cannot allocate device
+ * memory.  The paper has no counterpart: this is a deployment variant.
+ *   Some callers have no way to provide scratch: a plugin loaded into a host
+ *   program that owns all device memory and exposes no allocator, or a
+ *   latency-critical serving loop where a cudaMalloc (which can synchronise
+ *   the whole device) is not allowed.  This entry point takes the same
+ *   inputs and output as hca_decode but no workspace; its scratch lives in
+ *   one fixed device array inside the library (224 split slots of 131,584
+ *   bytes plus a small index: about 29.5 MB), which every GPU that loads the
+ *   library keeps until the process exits.
+ *   Limits: S <= HCA_NOALLOC_MAX_SEQS (64); larger S returns
+ *   HCA_ERR_UNSUPPORTED without launching.  The split uses at most
+ *   HCA_NOALLOC_MAX_CTAS (160) CTAs.
+ *   Set-up: the first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *   first call outside any stream capture.  Nothing is allocated, ever.
+ *   Sharing: every call uses the same array.  Nothing in it needs to start at
+ *   zero (each call writes every scratch value it later reads), but two calls
+ *   that overlap on the GPU (other streams, other threads) race on it:
+ *   serialise them.
+ */
+#define HCA_NOALLOC_MAX_SEQS 64
+#define HCA_NOALLOC_MAX_CTAS 160
+hca_status_t hca_decode_noalloc(const hca_bf16* q, const hca_bf16* ck, const hca_bf16* cv,
+                                int max_nc, const hca_bf16* wk, const hca_bf16* wv,
+                                const int32_t* ctx_len, const hca_bf16* g, int S, int H,
+                                float scale, hca_bf16* out, hca_stream_t stream);
+
+/*
  * hca_get_device_error — synchronises `stream`, then reads and clears the
  * device-side error word of the current device.  Returns HCA_OK,
  * HCA_ERR_TIMEOUT, HCA_ERR_DEVICE_INPUT or HCA_ERR_CUDA.  `where`, if not
