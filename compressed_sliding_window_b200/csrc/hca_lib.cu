@@ -14,7 +14,7 @@
 #include "../../include/hca.h"
 #include "hca_ptx.cuh"
 #include "compress.cuh"
-#include "prefill.cuh"
+#include "prefill2.cuh"
 #include "decode.cuh"
 
 namespace {
@@ -54,6 +54,52 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t X, uint64_t Y, uint64_t
              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 4-D view (64, Y, 8, W) of a [W][Y][512] bf16 tensor: x = element inside a
+// 64-wide column slab, y = row, z = slab index, w = batch.  A box
+// (64, box_y, box_z, 1) lands in shared memory as box_z slabs of
+// [box_y rows][64], each 128B-swizzled.
+bool make_map4(CUtensorMap* m, const void* base, uint64_t Y, uint64_t W, uint32_t box_y,
+               uint32_t box_z) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[4] = {64, Y, 8, W};
+  const cuuint64_t strides[3] = {1024, 128, Y * 1024};
+  const cuuint32_t box[4] = {64, box_y, box_z, 1};
+  const cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// How many 2-CTA clusters of the prefill kernel fit on the device at once.
+int prefill_max_pairs() {
+  static int cached = -1;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached > 0) return cached;
+  namespace P = hca::prefill2;
+  if (cudaFuncSetAttribute(P::prefill2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           P::kSmemAlloc) != cudaSuccess)
+    return -1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(P::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = P::kSmemAlloc;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 2;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, P::prefill2_kernel, &cfg) != cudaSuccess || n <= 0)
+    return -1;
+  cached = n;
+  return cached;
 }
 
 hca_status_t launch_status() {
@@ -104,7 +150,7 @@ hca_status_t hca_prefill_fwd(const hca_bf16* q, const hca_bf16* k, const hca_bf1
                              const hca_bf16* ck, const hca_bf16* cv, const hca_bf16* g, int B,
                              int T, int H, float scale, hca_bf16* out, float* lse,
                              hca_stream_t stream) {
-  namespace P = hca::prefill;
+  namespace P = hca::prefill2;
   if (H != HCA_NUM_HEADS) return HCA_ERR_UNSUPPORTED;
   if (B < 1 || T < 1 || !scale_ok(scale)) return HCA_ERR_INVALID_ARG;
   if (q == nullptr || k == nullptr || v == nullptr || g == nullptr || out == nullptr)
@@ -119,21 +165,20 @@ hca_status_t hca_prefill_fwd(const hca_bf16* q, const hca_bf16* k, const hca_bf1
   const long long items = static_cast<long long>(B) * row_tiles * 2;
   if (items > 0x7fffffffLL) return HCA_ERR_UNSUPPORTED;
 
+  const long long items2 = static_cast<long long>(B) * row_tiles;
+  if (items2 > 0x7fffffffLL) return HCA_ERR_UNSUPPORTED;
+  (void)items;
+
   P::Maps maps;
   const uint64_t rows = static_cast<uint64_t>(T) * HCA_NUM_HEADS;
-  bool ok = make_map(&maps.q, q, HCA_HEAD_DIM, rows, B, 128) &&
-            make_map(&maps.g, g, HCA_HEAD_DIM, rows, B, 128) &&
-            make_map(&maps.out, out, HCA_HEAD_DIM, rows, B, 128) &&
-            make_map(&maps.k, k, HCA_HEAD_DIM, T, B, 128) &&
-            make_map(&maps.v, v, HCA_HEAD_DIM, T, B, 128) &&
-            make_map(&maps.k16, k, HCA_HEAD_DIM, T, B, 16) &&
-            make_map(&maps.v16, v, HCA_HEAD_DIM, T, B, 16);
+  bool ok = make_map4(&maps.q4, q, rows, B, 128, 4) && make_map4(&maps.g4, g, rows, B, 128, 2) &&
+            make_map4(&maps.out4, out, rows, B, 128, 2) &&
+            make_map(&maps.kwin, k, HCA_HEAD_DIM, T, B, P::kWinN) &&
+            make_map4(&maps.v4, v, T, B, 64, 4);
   if (ok && nb > 0) {
-    ok = make_map(&maps.ck, ck, HCA_HEAD_DIM, nb, B, 128) &&
-         make_map(&maps.cv, cv, HCA_HEAD_DIM, nb, B, 128);
-  } else if (ok) {  // no compressed entry exists; the maps are never used
-    maps.ck = maps.k;
-    maps.cv = maps.v;
+    ok = make_map(&maps.ck, ck, HCA_HEAD_DIM, nb, B, P::kKT) && make_map4(&maps.cv4, cv, nb, B, 64, 4);
+  } else if (ok) {  // no compressed entry exists; these maps are never used
+    ok = make_map(&maps.ck, k, HCA_HEAD_DIM, T, B, P::kKT) && make_map4(&maps.cv4, v, T, B, 64, 4);
   }
   if (!ok) return HCA_ERR_CUDA;
 
@@ -141,16 +186,13 @@ hca_status_t hca_prefill_fwd(const hca_bf16* q, const hca_bf16* k, const hca_bf1
   prm.B = B;
   prm.T = T;
   prm.row_tiles = static_cast<int>(row_tiles);
-  prm.items = static_cast<int>(items);
+  prm.items = static_cast<int>(items2);
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.lse = lse;
-  const int sms = device_sms();
-  if (sms <= 0) return HCA_ERR_CUDA;
-  const int grid = static_cast<int>(items < sms ? items : sms);
-  if (cudaFuncSetAttribute(P::prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           P::kSmemAlloc) != cudaSuccess)
-    return HCA_ERR_CUDA;
-  P::prefill_kernel<<<grid, P::kThreads, P::kSmemAlloc, stream>>>(maps, prm);
+  const int max_pairs = prefill_max_pairs();
+  if (max_pairs <= 0) return HCA_ERR_CUDA;
+  const int pairs = static_cast<int>(items2 < max_pairs ? items2 : max_pairs);
+  P::prefill2_kernel<<<2 * pairs, P::kThreads, P::kSmemAlloc, stream>>>(maps, prm);
   return launch_status();
 }
 

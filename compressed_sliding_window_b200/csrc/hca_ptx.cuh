@@ -18,6 +18,7 @@ enum : unsigned {
   DEVERR_NONE = 0,
   DEVERR_TIMEOUT = 1u << 0,     // an mbarrier wait exceeded its limit
   DEVERR_BAD_INPUT = 1u << 1,   // a device-resident argument was out of range
+  DEVERR_LAYOUT = 1u << 2,      // shared memory was not placed as the kernel requires
 };
 
 __device__ unsigned int g_error_word;
@@ -98,8 +99,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
                                                volatile int* abort_flag, uint64_t limit_ns,
                                                unsigned where) {
-  const bool ok = mbar_wait(bar, parity, abort_flag, limit_ns, where);
-  return __all_sync(0xffffffffu, ok);
+  // only lane 0 polls; the others then take the (already completed) phase
+  // with one try_wait each, which gives every lane its own acquire
+  bool ok = true;
+  if ((threadIdx.x & 31u) == 0) ok = mbar_wait(bar, parity, abort_flag, limit_ns, where);
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  if (ok) mbar_try_wait(bar, parity);
+  return ok;
 }
 
 // ---------------------------------------------------------------------------
@@ -359,6 +365,16 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
   }
 }
 
+__device__ __forceinline__ bool mbar_wait_cluster_warp(uint32_t bar, uint32_t parity,
+                                                       volatile int* abort_flag, uint64_t limit_ns,
+                                                       unsigned where) {
+  bool ok = true;
+  if ((threadIdx.x & 31u) == 0) ok = mbar_wait_cluster(bar, parity, abort_flag, limit_ns, where);
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  if (ok) mbar_try_wait_acq_cluster(bar, parity);
+  return ok;
+}
+
 __device__ __forceinline__ void fence_proxy_async_all() {
   asm volatile("fence.proxy.async;" ::: "memory");
 }
@@ -393,6 +409,17 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// logistic sigmoid as 0.5 + 0.5 * tanh(x / 2): one MUFU op
+__device__ __forceinline__ float sigmoid_fast(float x) {
+  return fmaf(0.5f, tanh_approx(0.5f * x), 0.5f);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
