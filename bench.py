@@ -455,6 +455,35 @@ def bench_decode(cfg, dev, peaks, args):
     return res
 
 
+def run_profile_case(args):
+    """A few launches of one kernel family on a small synthetic case, for ncu
+    captures (--profile-case prefill:T or decode:S:L).  Inputs are drawn on the
+    device; nothing is timed or printed but a status line."""
+    import torch
+    import compressed_sliding_window_b200 as hca
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(0)
+    kind, *dims = args.profile_case.split(":")
+    rnd = lambda *shape, s=1.0: (torch.randn(shape, device=dev, generator=g) * s).to(torch.bfloat16)  # noqa: E731
+    if kind == "prefill":
+        T = int(dims[0])
+        q, gg, k, v, s = rnd(1, T, 64, 512), rnd(1, T, 64, 512), rnd(1, T, 512, s=0.5), rnd(1, T, 512), rnd(1, T)
+        for _ in range(args.warmup):
+            hca.forward(q, k, v, s, gg)
+    elif kind == "decode":
+        S, L = int(dims[0]), int(dims[1])
+        nc = L // 128
+        ck, cv = rnd(S, nc, 512), rnd(S, nc, 512)
+        wk, wv, q, gg = rnd(S, 128, 512), rnd(S, 128, 512), rnd(S, 64, 512), rnd(S, 64, 512)
+        ctx = torch.full((S,), L, dtype=torch.int32, device=dev)
+        for _ in range(args.warmup):
+            hca.decode(q, ck, cv, wk, wv, ctx, gg)
+    else:
+        raise SystemExit(f"unknown profile case {args.profile_case}")
+    torch.cuda.synchronize()
+    print("profile case done, device error", hca.device_error()[0])
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -502,9 +531,13 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=20)
     ap.add_argument("--steps-128k", type=int, default=10)
     ap.add_argument("--ref-positions", type=int, default=24)
+    ap.add_argument("--profile-case", default=None,
+                    help="prefill:T or decode:S:L -- a few untimed launches for ncu")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
-    if args.impl == "reference":
+    if args.profile_case:
+        run_profile_case(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
