@@ -34,17 +34,18 @@ constexpr int kHeads = 64;
 constexpr int kDim = 512;
 constexpr int kKeyTile = 128;
 constexpr int kWin = 128;
-constexpr int kStages = 8;
+constexpr int kStages = 4;
 constexpr int kSlab = 16384;        // [128 keys x 64 bf16] swizzled
+constexpr int kStage = 2 * kSlab;   // one copy: two 64-wide slabs of a 128-key tile
 constexpr int kQSlab = 8192;        // [64 heads x 64 bf16] swizzled
 constexpr int kSmemQ = 0;           // 8 x 8 KB
-constexpr int kSmemRing = 65536;    // 8 x 16 KB
-constexpr int kSmemPT = kSmemRing + kStages * kSlab;  // P^T [128 keys x 64 heads] bf16, 16 KB
+constexpr int kSmemRing = 65536;    // 4 x 32 KB
+constexpr int kSmemPT = kSmemRing + kStages * kStage;  // P^T [128 keys x 64 heads] bf16, 16 KB
 constexpr int kSmemRed = kSmemPT + 16384;             // reductions, 4 KB
 constexpr int kSmemBar = kSmemRed + 4096;
 constexpr int kSmemBytes = kSmemBar + 256;
 constexpr int kSmemAlloc = kSmemBytes + 1024;
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;
 constexpr float kTau = 8.0f;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kMaxSeqs = 8192;      // prefix sums kept in shared memory? no: global scan, see below
@@ -96,6 +97,7 @@ __device__ __forceinline__ int nc_of_len(int L) { return L >= 128 ? (L - 128) / 
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) plan_kernel(const int* __restrict__ ctx_len, int S,
                                                     int max_nc, long long* __restrict__ seq_tile) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __shared__ long long carry;
   __shared__ long long wsum[32];
   if (threadIdx.x == 0) carry = 0;
@@ -161,13 +163,24 @@ __device__ __forceinline__ int find_seq(const long long* seq_tile, int S, long l
   return lo;
 }
 
+// 4-D views (64, rows, 8 slabs, S) of [S][rows][512] tensors: a box
+// (64, rows, n, 1) lands as n 64-wide slabs of [rows][64], 128B-swizzled.
 struct Maps {
-  CUtensorMap q;    // [1][S*64][512], box 64 x 64
-  CUtensorMap ck;   // [S][max_nc][512], box 64 x 128
+  CUtensorMap q;    // (64, S*64, 8, 1),  box (64, 64, 8, 1): the whole q of one sequence
+  CUtensorMap ck;   // (64, max_nc, 8, S), box (64, 128, 2, 1)
   CUtensorMap cv;
-  CUtensorMap wk;   // [S][128][512], box 64 x 128
+  CUtensorMap wk;   // (64, 128, 8, S),   box (64, 128, 2, 1)
   CUtensorMap wv;
 };
+
+__device__ __forceinline__ void tma_load_4d_dec(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                                int x, int y, int z, int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar)
+      : "memory");
+}
 
 // Transpose-reduce of 64 per-lane values across the 32 lanes of a warp: on
 // return a[0], a[1] hold the reduction over all lanes for heads 2*lane and
@@ -204,6 +217,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // The plan kernel may still be running (programmatic dependent launch):
+  // wait for its results, then let the combine kernel launch early.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const long long N = p.seq_tile[p.S];
   const long long A0 = N * blockIdx.x / gridDim.x;
   const long long A1 = N * (blockIdx.x + 1) / gridDim.x;
@@ -235,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&maps.wk);
     tma_prefetch_desc(&maps.wv);
   }
-  if (warp == 1) {
+  if (warp == 2) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
     tc_fence_before();
@@ -247,18 +264,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Segments: maximal runs of this CTA's tiles inside one sequence.
   const int s_first = find_seq(p.seq_tile, p.S, A0);
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp <= 1) {
+    // ------------------------------------------------------------ producers
+    // Two warps alternate ring stages: one issuing thread cannot keep enough
+    // copies in flight to cover HBM latency.
     if (lane == 0) {
-      uint32_t ring = 0, quse = 0;
+      const int me = warp;
+      uint32_t u = 0, quse = 0;
       bool ok = true;
-      auto load = [&](const CUtensorMap* map, int x, int y, int z) -> bool {
-        const uint32_t st = ring % kStages;
-        if (!mbar_wait(bar(B_EMPTY + st), ((ring / kStages) & 1) ^ 1, abort_flag, kWaitLimitNs, 40))
-          return false;
-        mbar_expect_tx(bar(B_FULL + st), kSlab);
-        tma_load_3d(sRing + st * kSlab, map, bar(B_FULL + st), x, y, z);
-        ++ring;
+      auto load = [&](const CUtensorMap* map, int y, int z, int w) -> bool {
+        if ((u & 1) == static_cast<uint32_t>(me)) {
+          const uint32_t st = u % kStages;
+          if (!mbar_wait(bar(B_EMPTY + st), ((u / kStages) & 1) ^ 1, abort_flag, kWaitLimitNs, 40))
+            return false;
+          mbar_expect_tx(bar(B_FULL + st), kStage);
+          tma_load_4d_dec(sRing + st * kStage, map, bar(B_FULL + st), 0, y, z, w);
+        }
+        ++u;
         return true;
       };
       long long x = A0;
@@ -267,20 +289,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const long long seg_end = min(A1, p.seq_tile[s + 1]);
         const int j0 = static_cast<int>(x - p.seq_tile[s]);
         const int j1 = static_cast<int>(seg_end - p.seq_tile[s]);
-        ok = mbar_wait(bar(B_QEMPTY), (quse & 1) ^ 1, abort_flag, kWaitLimitNs, 41);
-        if (!ok) break;
-        mbar_expect_tx(bar(B_QFULL), 8 * kQSlab);
-        for (int d = 0; d < 8; ++d)
-          tma_load_3d(sQ + d * kQSlab, &maps.q, bar(B_QFULL), 64 * d, s * kHeads, 0);
+        if (me == 0) {
+          ok = mbar_wait(bar(B_QEMPTY), (quse & 1) ^ 1, abort_flag, kWaitLimitNs, 41);
+          if (!ok) break;
+          mbar_expect_tx(bar(B_QFULL), 8 * kQSlab);
+          tma_load_4d_dec(sQ, &maps.q, bar(B_QFULL), 0, s * kHeads, 0, 0);
+        }
         ++quse;
         auto load_k = [&](int j) -> bool {
-          for (int d = 0; d < 8 && ok; ++d)
-            ok = (j < si.nct) ? load(&maps.ck, 64 * d, j * kKeyTile, s) : load(&maps.wk, 64 * d, 0, s);
+          for (int d = 0; d < 4 && ok; ++d)
+            ok = (j < si.nct) ? load(&maps.ck, j * kKeyTile, 2 * d, s) : load(&maps.wk, 0, 2 * d, s);
           return ok;
         };
         auto load_v = [&](int j) -> bool {
-          for (int e = 0; e < 8 && ok; ++e)
-            ok = (j < si.nct) ? load(&maps.cv, 64 * e, j * kKeyTile, s) : load(&maps.wv, 64 * e, 0, s);
+          for (int e = 0; e < 4 && ok; ++e)
+            ok = (j < si.nct) ? load(&maps.cv, j * kKeyTile, 2 * e, s) : load(&maps.wv, 0, 2 * e, s);
           return ok;
         };
         if (!load_k(j0)) break;
@@ -291,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         x = seg_end;
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 2) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       uint32_t ring = 0, quse = 0, sidx = 0, pvidx = 0, nseg = 0;
@@ -304,16 +327,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           return false;
         tc_fence_after();
         const uint32_t dS = tmem + (buf ? kTmemS1 : kTmemS0);
-        for (int d = 0; d < 8; ++d) {
+        for (int d2 = 0; d2 < 4; ++d2) {
           const uint32_t st = ring % kStages;
           if (!mbar_wait(bar(B_FULL + st), (ring / kStages) & 1, abort_flag, kWaitLimitNs, 51))
             return false;
           tc_fence_after();
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t ad = sdesc_sw128(sRing + st * kSlab + 32 * k, 16, 1024);
-            const uint64_t bd = sdesc_sw128(sQ + d * kQSlab + 32 * k, 16, 1024);
-            umma_bf16(dS, ad, bd, idesc_s, (d | k) != 0);
+          for (int sl = 0; sl < 2; ++sl) {
+            const int d = 2 * d2 + sl;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint64_t ad = sdesc_sw128(sRing + st * kStage + sl * kSlab + 32 * k, 16, 1024);
+              const uint64_t bd = sdesc_sw128(sQ + d * kQSlab + 32 * k, 16, 1024);
+              umma_bf16(dS, ad, bd, idesc_s, (d | k) != 0);
+            }
           }
           umma_commit(bar(B_EMPTY + st));
           ++ring;
@@ -328,22 +355,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           return false;
         tc_fence_after();
         for (int c = 0; c < 4; ++c) {
-          const uint32_t stA = ring % kStages, stB = (ring + 1) % kStages;
-          if (!mbar_wait(bar(B_FULL + stA), (ring / kStages) & 1, abort_flag, kWaitLimitNs, 54))
-            return false;
-          if (!mbar_wait(bar(B_FULL + stB), ((ring + 1) / kStages) & 1, abort_flag, kWaitLimitNs,
-                         55))
+          const uint32_t st = ring % kStages;
+          if (!mbar_wait(bar(B_FULL + st), (ring / kStages) & 1, abort_flag, kWaitLimitNs, 54))
             return false;
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
-            const uint64_t ad = sdesc_sw128(sRing + stA * kSlab + 2048 * k, kSlab, 1024);
+            const uint64_t ad = sdesc_sw128(sRing + st * kStage + 2048 * k, kSlab, 1024);
             const uint64_t bd = sdesc_sw128(sPT + 2048 * k, kSlab, 1024);
             umma_bf16(tmem + kTmemO + 64 * c, ad, bd, idesc_o, (!first || k > 0) ? 1u : 0u);
           }
-          umma_commit(bar(B_EMPTY + stA));
-          umma_commit(bar(B_EMPTY + stB));
-          ring += 2;
+          umma_commit(bar(B_EMPTY + st));
+          ++ring;
         }
         umma_commit(bar(B_PFREE));
         ++pvidx;
@@ -376,9 +399,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax / partial epilogue
-    const int tid = threadIdx.x - 64;        // 0..127
+    const int tid = threadIdx.x - 96;        // 0..127
     const int wq = warp & 3;
-    const int gw = warp - 2;                 // 0..3 within the group
+    const int gw = warp - 3;                 // 0..3 within the group
     const int key = wq * 32 + lane;          // TMEM lane == key row of S^T / dv row of O^T
     const uint32_t tl = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     uint32_t sidx = 0, pvidx = 0, nseg = 0;
@@ -532,20 +555,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
 }
 
 // ---------------------------------------------------------------------------
-// Combine: one CTA per (sequence, head); 128 threads x 4 dv.
+// Combine: CTA (sequence s, 8 heads), one warp per head, 16 value columns per
+// lane.  The weights 2^(m_c - M) of all partials are computed in parallel
+// across lanes and broadcast with shuffles, so the partial rows stream with
+// independent loads.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(128)
+constexpr int kCombineHeads = 8;
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(32 * kCombineHeads)
     combine_kernel(const Params p, int grid, const uint16_t* __restrict__ g,
                    uint16_t* __restrict__ out) {
+  pdl_wait();  // the split pass (a prerequisite grid) has finished and its writes are visible
   const int s = blockIdx.x;
-  const int h = blockIdx.y;
+  const int h = blockIdx.y * kCombineHeads + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
   const long long N = p.seq_tile[p.S];
   const long long P0 = p.seq_tile[s], P1 = p.seq_tile[s + 1];
   // CTA that owns global tile x: ceil((x + 1) * grid / N) - 1
@@ -553,38 +588,68 @@ __global__ void __launch_bounds__(128)
     return static_cast<int>(((x + 1) * grid + N - 1) / N) - 1;
   };
   const int c0 = owner(P0), c1 = owner(P1 - 1);
+  const int np = c1 - c0 + 1;
+  auto nonempty = [&](int c) { return N * c / grid < N * (c + 1) / grid; };
+  // pass 1: M = max of the partial maxima
   float M = -INFINITY;
-  for (int c = c0; c <= c1; ++c) {
-    if (N * c / grid >= N * (c + 1) / grid) continue;
-    M = fmaxf(M, p.ws_ml[static_cast<size_t>(c + s) * 128 + h]);
+  for (int base = 0; base < np; base += 32) {
+    const int c = c0 + base + lane;
+    if (base + lane < np && nonempty(c))
+      M = fmaxf(M, p.ws_ml[static_cast<size_t>(c + s) * 128 + h]);
   }
-  const float Mu = (M == -INFINITY) ? 0.f : M;
-  float Lsum = 0.f;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int c = c0; c <= c1; ++c) {
-    if (N * c / grid >= N * (c + 1) / grid) continue;
-    const size_t slot = static_cast<size_t>(c + s);
-    const float w = ex2_approx(p.ws_ml[slot * 128 + h] - Mu);
-    Lsum += w * p.ws_ml[slot * 128 + 64 + h];
-    const float4 o = *reinterpret_cast<const float4*>(p.ws_o + (slot * kHeads + h) * kDim +
-                                                      4 * threadIdx.x);
-    acc[0] += w * o.x;
-    acc[1] += w * o.y;
-    acc[2] += w * o.z;
-    acc[3] += w * o.w;
-  }
-  const float inv = 1.f / Lsum;
-  const size_t base = (static_cast<size_t>(s) * kHeads + h) * kDim + 4 * threadIdx.x;
-  const uint2 gv = *reinterpret_cast<const uint2*>(g + base);
-  const float gf[4] = {bf16lo_to_f32(gv.x), bf16hi_to_f32(gv.x), bf16lo_to_f32(gv.y),
-                       bf16hi_to_f32(gv.y)};
-  float r[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float sg = 1.f / (1.f + ex2_approx(-1.4426950408889634f * gf[i]));
-    r[i] = acc[i] * inv * sg;
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const float Mu = (M == -INFINITY) ? 0.f : M;
+  // pass 2: weighted sum of the partial rows and of their denominators
+  float acc[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+  float L = 0.f;
+  for (int base = 0; base < np; base += 32) {
+    const int c = c0 + base + lane;
+    float w = 0.f, lw = 0.f;
+    if (base + lane < np && nonempty(c)) {
+      const size_t slot = static_cast<size_t>(c + s);
+      w = ex2_approx(p.ws_ml[slot * 128 + h] - Mu);
+      lw = w * p.ws_ml[slot * 128 + 64 + h];
+    }
+    L += lw;
+    const int cnt = min(32, np - base);
+    for (int i = 0; i < cnt; ++i) {
+      const float wi = __shfl_sync(0xffffffffu, w, i);
+      if (wi == 0.f) continue;  // empty split (or a fully masked one)
+      const size_t slot = static_cast<size_t>(c0 + base + i + s);
+      const float4* src = reinterpret_cast<const float4*>(p.ws_o + (slot * kHeads + h) * kDim) +
+                          lane * 4;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 o = __ldg(src + q);
+        acc[4 * q + 0] = fmaf(wi, o.x, acc[4 * q + 0]);
+        acc[4 * q + 1] = fmaf(wi, o.y, acc[4 * q + 1]);
+        acc[4 * q + 2] = fmaf(wi, o.z, acc[4 * q + 2]);
+        acc[4 * q + 3] = fmaf(wi, o.w, acc[4 * q + 3]);
+      }
+    }
   }
-  *reinterpret_cast<uint2*>(out + base) = make_uint2(pack_bf16x2(r[0], r[1]), pack_bf16x2(r[2], r[3]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+  const float inv = 1.f / L;
+  const size_t base = (static_cast<size_t>(s) * kHeads + h) * kDim + 16 * lane;
+  const uint4* gp = reinterpret_cast<const uint4*>(g + base);
+  uint4* op = reinterpret_cast<uint4*>(out + base);
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const uint4 gv = __ldg(gp + q);
+    const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+    uint32_t ow[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float a0 = acc[8 * q + 2 * k] * inv * sigmoid_fast(bf16lo_to_f32(gw[k]));
+      const float a1 = acc[8 * q + 2 * k + 1] * inv * sigmoid_fast(bf16hi_to_f32(gw[k]));
+      ow[k] = pack_bf16x2(a0, a1);
+    }
+    op[q] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+  }
 }
 
 }  // namespace decode

@@ -10,6 +10,7 @@
 #include <cmath>
 #include <cstdint>
 #include <mutex>
+#include <utility>
 
 #include "../../include/hca.h"
 #include "hca_ptx.cuh"
@@ -100,6 +101,25 @@ int prefill_max_pairs() {
     return -1;
   cached = n;
   return cached;
+}
+
+// Launch `kernel` on `stream` allowing programmatic dependent launch: it may
+// start while the previous kernel on the stream is still running, and waits
+// for it inside (griddepcontrol.wait).
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 hca_status_t launch_status() {
@@ -238,12 +258,11 @@ hca_status_t hca_decode(const hca_bf16* q, const hca_bf16* ck, const hca_bf16* c
   prm.seq_tile = reinterpret_cast<long long*>(wsb + ((D::ws_bytes(slots) + 255) & ~size_t(255)));
 
   D::Maps maps;
-  bool ok = make_map(&maps.q, q, HCA_HEAD_DIM, static_cast<uint64_t>(S) * HCA_NUM_HEADS, 1, 64) &&
-            make_map(&maps.wk, wk, HCA_HEAD_DIM, HCA_WINDOW, S, 128) &&
-            make_map(&maps.wv, wv, HCA_HEAD_DIM, HCA_WINDOW, S, 128);
+  bool ok = make_map4(&maps.q, q, static_cast<uint64_t>(S) * HCA_NUM_HEADS, 1, 64, 8) &&
+            make_map4(&maps.wk, wk, HCA_WINDOW, S, 128, 2) &&
+            make_map4(&maps.wv, wv, HCA_WINDOW, S, 128, 2);
   if (ok && max_nc > 0) {
-    ok = make_map(&maps.ck, ck, HCA_HEAD_DIM, max_nc, S, 128) &&
-         make_map(&maps.cv, cv, HCA_HEAD_DIM, max_nc, S, 128);
+    ok = make_map4(&maps.ck, ck, max_nc, S, 128, 2) && make_map4(&maps.cv, cv, max_nc, S, 128, 2);
   } else if (ok) {
     maps.ck = maps.wk;
     maps.cv = maps.wv;
@@ -255,9 +274,12 @@ hca_status_t hca_decode(const hca_bf16* q, const hca_bf16* ck, const hca_bf16* c
   if (cudaFuncSetAttribute(D::decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            D::kSmemAlloc) != cudaSuccess)
     return HCA_ERR_CUDA;
-  D::decode_kernel<<<sms, D::kThreads, D::kSmemAlloc, stream>>>(maps, prm);
-  if (cudaGetLastError() != cudaSuccess) return HCA_ERR_CUDA;
-  D::combine_kernel<<<dim3(S, HCA_NUM_HEADS), 128, 0, stream>>>(prm, sms, g, out);
+  if (launch_pdl(D::decode_kernel, dim3(sms), dim3(D::kThreads), D::kSmemAlloc, stream, maps,
+                 prm) != cudaSuccess)
+    return HCA_ERR_CUDA;
+  if (launch_pdl(D::combine_kernel, dim3(S, HCA_NUM_HEADS / D::kCombineHeads),
+                 dim3(32 * D::kCombineHeads), 0, stream, prm, sms, g, out) != cudaSuccess)
+    return HCA_ERR_CUDA;
   return launch_status();
 }
 
@@ -335,12 +357,11 @@ hca_status_t hca_decode_noalloc(const hca_bf16* q, const hca_bf16* ck, const hca
   prm.seq_tile = reinterpret_cast<long long*>(wsb + kNoAllocPrefixOffset);
 
   D::Maps maps;
-  bool ok = make_map(&maps.q, q, HCA_HEAD_DIM, static_cast<uint64_t>(S) * HCA_NUM_HEADS, 1, 64) &&
-            make_map(&maps.wk, wk, HCA_HEAD_DIM, HCA_WINDOW, S, 128) &&
-            make_map(&maps.wv, wv, HCA_HEAD_DIM, HCA_WINDOW, S, 128);
+  bool ok = make_map4(&maps.q, q, static_cast<uint64_t>(S) * HCA_NUM_HEADS, 1, 64, 8) &&
+            make_map4(&maps.wk, wk, HCA_WINDOW, S, 128, 2) &&
+            make_map4(&maps.wv, wv, HCA_WINDOW, S, 128, 2);
   if (ok && max_nc > 0) {
-    ok = make_map(&maps.ck, ck, HCA_HEAD_DIM, max_nc, S, 128) &&
-         make_map(&maps.cv, cv, HCA_HEAD_DIM, max_nc, S, 128);
+    ok = make_map4(&maps.ck, ck, max_nc, S, 128, 2) && make_map4(&maps.cv, cv, max_nc, S, 128, 2);
   } else if (ok) {
     maps.ck = maps.wk;
     maps.cv = maps.wv;
@@ -352,9 +373,12 @@ hca_status_t hca_decode_noalloc(const hca_bf16* q, const hca_bf16* ck, const hca
   if (cudaFuncSetAttribute(D::decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            D::kSmemAlloc) != cudaSuccess)
     return HCA_ERR_CUDA;
-  D::decode_kernel<<<grid, D::kThreads, D::kSmemAlloc, stream>>>(maps, prm);
-  if (cudaGetLastError() != cudaSuccess) return HCA_ERR_CUDA;
-  D::combine_kernel<<<dim3(S, HCA_NUM_HEADS), 128, 0, stream>>>(prm, grid, g, out);
+  if (launch_pdl(D::decode_kernel, dim3(grid), dim3(D::kThreads), D::kSmemAlloc, stream, maps,
+                 prm) != cudaSuccess)
+    return HCA_ERR_CUDA;
+  if (launch_pdl(D::combine_kernel, dim3(S, HCA_NUM_HEADS / D::kCombineHeads),
+                 dim3(32 * D::kCombineHeads), 0, stream, prm, grid, g, out) != cudaSuccess)
+    return HCA_ERR_CUDA;
   return launch_status();
 }
 
