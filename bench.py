@@ -241,11 +241,12 @@ def run_ours(args):
     ck = torch.empty((B, nb, 512), dtype=torch.bfloat16, device=dev)
     cv = torch.empty_like(ck)
     out = torch.empty_like(d["q"])
+    ws = torch.empty((hca.prefill_workspace_size(B, T),), dtype=torch.uint8, device=dev)
     torch.cuda.synchronize()
 
     def step():
         hca.compress(d["k"], d["v"], d["s"], ck, cv)
-        hca.prefill(d["q"], d["k"], d["v"], ck, cv, d["g"], out=out)
+        hca.prefill(d["q"], d["k"], d["v"], ck, cv, d["g"], out=out, workspace=ws)
 
     for _ in range(args.warmup):
         step()
@@ -268,7 +269,7 @@ def run_ours(args):
     for i in range(args.steps):
         hca.compress(d["k"], d["v"], d["s"], ck, cv)
         ev[i][0].record(stream)
-        hca.prefill(d["q"], d["k"], d["v"], ck, cv, d["g"], out=out)
+        hca.prefill(d["q"], d["k"], d["v"], ck, cv, d["g"], out=out, workspace=ws)
         ev[i][1].record(stream)
     t_end.record(stream)
     barrier(world)
@@ -283,7 +284,7 @@ def run_ours(args):
     value = job_throughput(flops, world, args.steps, max_ms) / 1e12
     alg_bytes = prefill_bytes(B, T)
     achieved_gbs = alg_bytes / (prefill_ms / 1e3) / 1e9
-    traffic = read_traffic("prefill.cuh", "prefill_T32768_traffic.txt")
+    traffic = read_traffic("prefill2.cuh", "prefill2_T32768_traffic.txt")
     result = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
@@ -293,7 +294,7 @@ def run_ours(args):
                                "1 KV head, block 128, window 128",
                    "global_batch": world * B, "seq_len": T, "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2 (4.3 GB read per step)"},
-        "roofline": {"kernel": "prefill_kernel", "bound": "hbm", "achieved": achieved_gbs,
+        "roofline": {"kernel": "prefill2_kernel", "bound": "hbm", "achieved": achieved_gbs,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved_gbs / peaks["hbm_gbs"],
                      "traffic": traffic, "peak_source": peaks["source"],
@@ -315,7 +316,7 @@ def run_ours(args):
         for n in d:
             d[n].copy_(hx[n], non_blocking=True)
         hca.compress(d["k"], d["v"], d["s"], ck, cv)
-        hca.prefill(d["q"], d["k"], d["v"], ck, cv, d["g"], out=out)
+        hca.prefill(d["q"], d["k"], d["v"], ck, cv, d["g"], out=out, workspace=ws)
         hout.copy_(out, non_blocking=True)
 
     e2e_step()
@@ -361,9 +362,10 @@ def bench_prefill_128k(dev, peaks, args):
     ck = torch.empty((1, nb, 512), dtype=torch.bfloat16, device=dev)
     cv = torch.empty_like(ck)
     out = torch.empty_like(d["q"])
+    ws = torch.empty((hca.prefill_workspace_size(1, T),), dtype=torch.uint8, device=dev)
     for _ in range(3):
         hca.compress(d["k"], d["v"], d["s"], ck, cv)
-        hca.prefill(d["q"], d["k"], d["v"], ck, cv, d["g"], out=out)
+        hca.prefill(d["q"], d["k"], d["v"], ck, cv, d["g"], out=out, workspace=ws)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream(dev)
     n = args.steps_128k
@@ -372,7 +374,7 @@ def bench_prefill_128k(dev, peaks, args):
     for i in range(n):
         hca.compress(d["k"], d["v"], d["s"], ck, cv)
         ev[i][0].record(stream)
-        hca.prefill(d["q"], d["k"], d["v"], ck, cv, d["g"], out=out)
+        hca.prefill(d["q"], d["k"], d["v"], ck, cv, d["g"], out=out, workspace=ws)
         ev[i][1].record(stream)
     torch.cuda.synchronize()
     code, where = hca.device_error(dev)

@@ -48,7 +48,9 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
         L.hca_compress.argtypes = [vp, vp, vp, i, i, vp, vp, vp]
-        L.hca_prefill_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, f, vp, vp, vp]
+        L.hca_prefill_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, f, vp, vp, vp, sz, vp]
+        L.hca_prefill_workspace_size.argtypes = [i, i]
+        L.hca_prefill_workspace_size.restype = sz
         L.hca_decode_workspace_size.argtypes = [i]
         L.hca_decode_workspace_size.restype = sz
         L.hca_decode.argtypes = [vp, vp, vp, i, vp, vp, vp, vp, i, i, f, vp, sz, vp, vp]
@@ -114,9 +116,14 @@ def compress(k: torch.Tensor, v: torch.Tensor, s: torch.Tensor,
     return ck, cv
 
 
+def prefill_workspace_size(B: int, T: int) -> int:
+    return int(lib().hca_prefill_workspace_size(B, T))
+
+
 def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, ck: torch.Tensor,
             cv: torch.Tensor, g: torch.Tensor, scale: Optional[float] = None,
-            out: Optional[torch.Tensor] = None, return_lse: bool = False):
+            out: Optional[torch.Tensor] = None, return_lse: bool = False,
+            workspace: Optional[torch.Tensor] = None):
     """HCA prefill attention with the gate fused.
 
     q, g: [B, T, 64, 512]; k, v: [B, T, 512]; ck, cv: [B, T // 128, 512]
@@ -136,10 +143,14 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, ck: torch.Tensor,
         out = torch.empty_like(q)
     _check(out, "out", (B, T, H, HEAD_DIM))
     lse = torch.empty((B, T, H), dtype=torch.float32, device=q.device) if return_lse else None
+    if workspace is None:
+        workspace = torch.empty((prefill_workspace_size(B, T),), dtype=torch.uint8,
+                                device=q.device)
+    _check(workspace, "workspace", dtype=torch.uint8)
     _ok("hca_prefill_fwd", lib().hca_prefill_fwd(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(ck) if nb else None,
         _ptr(cv) if nb else None, g.data_ptr(), B, T, H, ctypes.c_float(scale), out.data_ptr(),
-        _ptr(lse), _stream(q.device)))
+        _ptr(lse), workspace.data_ptr(), workspace.numel(), _stream(q.device)))
     return (out, lse) if return_lse else out
 
 

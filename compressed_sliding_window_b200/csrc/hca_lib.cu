@@ -166,15 +166,26 @@ hca_status_t hca_compress(const hca_bf16* k, const hca_bf16* v, const hca_bf16* 
   return launch_status();
 }
 
+size_t hca_prefill_workspace_size(int B, int T) {
+  if (B < 1 || T < 1) return 0;
+  const long long items = static_cast<long long>(B) * ((T + 1) / 2);
+  const int max_pairs = prefill_max_pairs();
+  if (max_pairs <= 0) return 0;
+  const long long pairs = items < max_pairs ? items : max_pairs;
+  return static_cast<size_t>(pairs) * hca::prefill2::kScratchPerPair + 256;
+}
+
 hca_status_t hca_prefill_fwd(const hca_bf16* q, const hca_bf16* k, const hca_bf16* v,
                              const hca_bf16* ck, const hca_bf16* cv, const hca_bf16* g, int B,
-                             int T, int H, float scale, hca_bf16* out, float* lse,
-                             hca_stream_t stream) {
+                             int T, int H, float scale, hca_bf16* out, float* lse, void* ws,
+                             size_t ws_bytes, hca_stream_t stream) {
   namespace P = hca::prefill2;
   if (H != HCA_NUM_HEADS) return HCA_ERR_UNSUPPORTED;
   if (B < 1 || T < 1 || !scale_ok(scale)) return HCA_ERR_INVALID_ARG;
-  if (q == nullptr || k == nullptr || v == nullptr || g == nullptr || out == nullptr)
+  if (q == nullptr || k == nullptr || v == nullptr || g == nullptr || out == nullptr ||
+      ws == nullptr)
     return HCA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return HCA_ERR_INVALID_ARG;
   const int nb = T / HCA_BLOCK;
   if (nb > 0 && (ck == nullptr || cv == nullptr)) return HCA_ERR_INVALID_ARG;
   const void* ptrs[7] = {q, k, v, g, out, ck, cv};
@@ -196,9 +207,9 @@ hca_status_t hca_prefill_fwd(const hca_bf16* q, const hca_bf16* k, const hca_bf1
             make_map(&maps.kwin, k, HCA_HEAD_DIM, T, B, P::kWinN) &&
             make_map4(&maps.v4, v, T, B, 64, 4);
   if (ok && nb > 0) {
-    ok = make_map(&maps.ck, ck, HCA_HEAD_DIM, nb, B, P::kKT) && make_map4(&maps.cv4, cv, nb, B, 64, 4);
+    ok = make_map(&maps.ck, ck, HCA_HEAD_DIM, nb, B, 64) && make_map4(&maps.cv4, cv, nb, B, 64, 4);
   } else if (ok) {  // no compressed entry exists; these maps are never used
-    ok = make_map(&maps.ck, k, HCA_HEAD_DIM, T, B, P::kKT) && make_map4(&maps.cv4, v, T, B, 64, 4);
+    ok = make_map(&maps.ck, k, HCA_HEAD_DIM, T, B, 64) && make_map4(&maps.cv4, v, T, B, 64, 4);
   }
   if (!ok) return HCA_ERR_CUDA;
 
@@ -209,9 +220,11 @@ hca_status_t hca_prefill_fwd(const hca_bf16* q, const hca_bf16* k, const hca_bf1
   prm.items = static_cast<int>(items2);
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.lse = lse;
+  prm.pscratch = static_cast<uint8_t*>(ws);
   const int max_pairs = prefill_max_pairs();
   if (max_pairs <= 0) return HCA_ERR_CUDA;
   const int pairs = static_cast<int>(items2 < max_pairs ? items2 : max_pairs);
+  if (ws_bytes < static_cast<size_t>(pairs) * P::kScratchPerPair) return HCA_ERR_INVALID_ARG;
   P::prefill2_kernel<<<2 * pairs, P::kThreads, P::kSmemAlloc, stream>>>(maps, prm);
   return launch_status();
 }

@@ -76,9 +76,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Bounded wait for the phase with the given parity to complete.  Returns false
 // when the CTA-wide abort flag is raised or the limit runs out (the latter
 // raises the flag and records DEVERR_TIMEOUT with `where`).  Never spins forever.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          uint64_t limit_ns, unsigned where) {
-  if (mbar_try_wait(bar, parity)) return true;
+// The polling loop is out of line: the fast path (phase already complete) is
+// one try_wait at the call site, and the many call sites in the hot loops do
+// not each carry a copy of the loop (instruction-cache footprint).
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity,
+                                            volatile int* abort_flag, uint64_t limit_ns,
+                                            unsigned where) {
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -91,6 +94,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       }
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_ns, unsigned where) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort_flag, limit_ns, where);
 }
 
 // Warp-collective bounded wait: every lane of the warp gets the same answer,
@@ -149,6 +158,11 @@ __device__ __forceinline__ void bulk_commit() {
 }
 __device__ __forceinline__ void bulk_wait_read_all() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// wait until at most N of this thread's bulk groups still read their source
+template <int N>
+__device__ __forceinline__ void bulk_wait_read_n() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
 }
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
@@ -291,6 +305,19 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   return d;
 }
 
+// Shared-memory matrix descriptor for the no-swizzle K-major layout: 8-row x
+// 16-byte core matrices stored contiguously (128 B each); `lbo_bytes` is the
+// distance between core matrices along K, `sbo_bytes` along M/N.
+__device__ __forceinline__ uint64_t sdesc_noswz(uint32_t saddr, uint32_t lbo_bytes,
+                                                uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;
+  return d;
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 D:
 // D fmt F32=1 [4,6), A fmt BF16=1 [7,10), B fmt BF16=1 [10,13),
 // A major [15], B major [16] (0 = K-major, 1 = MN-major), N>>3 [17,23), M>>4 [24,29).
@@ -347,10 +374,9 @@ __device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint32_t bar, uint32_t
 
 // Bounded wait on a local mbarrier whose arrivals come from another CTA of
 // the cluster (acquire at cluster scope).
-__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
-                                                  volatile int* abort_flag, uint64_t limit_ns,
-                                                  unsigned where) {
-  if (mbar_try_wait_acq_cluster(bar, parity)) return true;
+static __device__ __noinline__ bool mbar_wait_cluster_slow(uint32_t bar, uint32_t parity,
+                                                    volatile int* abort_flag, uint64_t limit_ns,
+                                                    unsigned where) {
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait_acq_cluster(bar, parity)) return true;
@@ -363,6 +389,13 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
       }
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
+                                                  volatile int* abort_flag, uint64_t limit_ns,
+                                                  unsigned where) {
+  if (mbar_try_wait_acq_cluster(bar, parity)) return true;
+  return mbar_wait_cluster_slow(bar, parity, abort_flag, limit_ns, where);
 }
 
 __device__ __forceinline__ bool mbar_wait_cluster_warp(uint32_t bar, uint32_t parity,

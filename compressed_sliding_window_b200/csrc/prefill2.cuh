@@ -9,9 +9,13 @@
 // of an SM, so no single SM can hold O and the scores.  The cluster's two CTAs
 // split the work by operation instead of by value columns:
 //   rank 0, the S-CTA: Q resident in shared memory, S = Q K^T on tcgen05 into
-//     two 256-column TMEM buffers, the online softmax (thread = row), and P
-//     (bf16) shipped to rank 1's shared memory over DSMEM in 128-key sub-tiles
-//     together with the per-row rescale factor.
+//     two 256-column TMEM buffers, the online softmax, and P (bf16) in 128-key
+//     sub-tiles.  P does not go over DSMEM (its per-SM store rate is far below
+//     what a tile needs): the S-CTA writes each sub-tile to a small
+//     L2-resident scratch with plain global stores, already in the no-swizzle
+//     core-matrix layout the MMA reads (8-key chunk major, so the 32 rows of a
+//     warp store 512 contiguous bytes), and a warp of rank 1 pulls it with one
+//     bulk copy.  Only the per-row rescale factors cross over DSMEM.
 //   rank 1, the O-CTA: the full O (128 x 512 fp32) in TMEM, O += P V on
 //     tcgen05, the rare O rescale, and the epilogue out = O / l * sigmoid(g)
 //     (g staged by TMA, out written in place and TMA-stored).
@@ -29,12 +33,18 @@
 // brings 4 (V) or 2 (g) 64-wide column slabs, already in the layout the MMA
 // and the epilogue read.
 //
-// Warp roles (352 threads): warps 0-1 TMA producers, warp 2 MMA issuer and
+// Warp roles (416 threads): warps 0-1 TMA producers, warp 2 MMA issuer and
 // TMEM owner, warps 3-10 compute: two warps per TMEM lane quadrant, so a tile
 // row is shared by two threads.  On rank 0 each of them owns one 128-key half
 // of the score tile (= one P sub-tile; the row max is exchanged through shared
-// memory); on rank 1 each owns 256 of the 512 value columns (rescale and
-// epilogue).
+// memory under a 64-thread named barrier); on rank 1 they rescale O (each 256
+// of the 512 value columns) and run the epilogue (128 columns per stage).
+// Rank 1 also has warp 11, the P copier, and warp 12, which stores the
+// epilogue's output stages and hands them back to the producers.
+//
+// Code size.  The kernel is bound by instruction fetch long before its loops
+// are: every role's hot loop is kept small (32-column chunks, one code path
+// for masked and unmasked chunks, bounded waits polled out of line).
 #pragma once
 
 #include "hca_ptx.cuh"
@@ -46,7 +56,8 @@ constexpr int kRows = 128;
 constexpr int kHeads = 64;
 constexpr int kKT = 256;     // compressed key tile
 constexpr int kWinN = 144;   // raw key tile
-constexpr int kThreads = 352;
+constexpr int kThreads = 416;
+constexpr int kScratchPerPair = 4 * 32768;   // 2 tile parities x 2 sub-tiles
 constexpr float kTau = 8.0f;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
@@ -57,35 +68,40 @@ constexpr int S_KRING = 131072;              // 3 stages x [256 keys][64]
 constexpr int kKStages = 3;
 constexpr int kKStage = 32768;
 // ---- O-CTA shared memory
-constexpr int O_P = 0;                       // 2 sub-tile buffers x [2 slabs][128 rows][64 keys]
+constexpr int O_P = 0;                       // 2 sub-tile buffers x [16 key chunks][128 rows][8 keys]
 constexpr int kPBuf = 32768;
-constexpr int O_VRING = 65536;               // 4 stages x [4 slabs][64 keys][64 dv]
-constexpr int kVStages = 4;
+constexpr int O_VRING = 65536;               // 5 stages x [4 slabs][64 keys][64 dv]
+constexpr int kVStages = 5;
 constexpr int kVStage = 32768;
-constexpr int O_ALPHA = O_VRING + kVStages * kVStage;  // [128] float
-constexpr int O_FLAGS = O_ALPHA + 512;                  // [4] int
-constexpr int O_INVL = O_FLAGS + 64;                    // [128] float
 
 // ---- barriers (both CTAs, same offsets)
 constexpr int BAR = 229376;
 enum {
   QFULL = 0, QEMPTY = 2, KFULL = 4, KEMPTY = KFULL + kKStages, SFULL = KEMPTY + kKStages,
-  SFREE = SFULL + 2, PFREE = SFREE + 2, STATSFREE = PFREE + 2,
-  VFULL = STATSFREE + 1, VEMPTY = VFULL + kVStages, PFULL = VEMPTY + kVStages, CORR = PFULL + 2,
-  PVDONE = CORR + 1, OFULL = PVDONE + 1, OFREE = OFULL + 1, STATSFULL = OFREE + 1,
-  STAGED = STATSFULL + 1, DRAIN = STAGED + 2, XMAX = DRAIN + 1, NBAR = XMAX + 4
+  SFREE = SFULL + 2, PFREE = SFREE + 2, STATSFREE = PFREE + 4,
+  VFULL = STATSFREE + 1, VEMPTY = VFULL + kVStages, PREADY = VEMPTY + kVStages,
+  PFULL = PREADY + 4, PBUFFREE = PFULL + 2, CORR = PBUFFREE + 2,
+  PVDONE = CORR + 2, OFULL = PVDONE + 2, OFREE = OFULL + 1, STATSFULL = OFREE + 2,
+  STAGED = STATSFULL + 1, DRAIN = STAGED + 4, NBAR = DRAIN + 1
 };
 constexpr int kTmemSlot = BAR + 8 * NBAR;
 constexpr int kAbortSlot = kTmemSlot + 4;
 // S-CTA: per-row statistics exchanged between the two warps of a row
-// ([2 parity][2 halves][128] float)
+// ([2 parity][2 halves][128] float) and their ok flags ([2][2][4 quadrants] int)
 constexpr int S_XMAX = BAR + 512;
-constexpr int kSmemBytes = S_XMAX + 2048;
+constexpr int S_XOK = S_XMAX + 2048;
+// O-CTA: rescale factors [2 tile parities][128] float, rescale flags
+// [2 tile parities][4] int, 1/l [128] float
+constexpr int O_ALPHA = BAR + 512;
+constexpr int O_FLAGS = O_ALPHA + 1024;
+constexpr int O_INVL = O_FLAGS + 64;
+constexpr int kSmemBytes = S_XOK + 64;
 // The dynamic shared memory base is 1024-aligned (checked at run time), so no
 // alignment slack is allocated: the S-CTA needs every byte.
 constexpr int kSmemAlloc = kSmemBytes;
 static_assert(kAbortSlot + 4 <= kSmemBytes, "barrier region overflow");
-static_assert(O_INVL + 512 <= BAR, "O-CTA layout overflow");
+static_assert(O_VRING + kVStages * kVStage <= BAR, "O-CTA ring overflow");
+static_assert(O_INVL + 512 <= kSmemBytes, "O-CTA layout overflow");
 static_assert(S_KRING + kKStages * kKStage <= BAR, "S-CTA layout overflow");
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
 
@@ -95,11 +111,12 @@ struct Params {
   int items;        // B * row_tiles
   float scale_log2; // softmax scale * log2(e)
   float* lse;       // [B, T, 64] or null
+  uint8_t* pscratch;  // [pairs][4][32 KB] P sub-tile images
 };
 
 struct Maps {
   CUtensorMap q4;    // (64, T*64, 8, B)  box (64, 128, 4, 1): one Q half
-  CUtensorMap ck;    // [B][nb][512]      box (64, 256, 1)
+  CUtensorMap ck;    // [B][nb][512]      box (64, 64, 1): tiles load only the rows they use
   CUtensorMap kwin;  // [B][T][512]       box (64, 144, 1)
   CUtensorMap cv4;   // (64, nb, 8, B)    box (64, 64, 4, 1)
   CUtensorMap v4;    // (64, T, 8, B)     box (64, 64, 4, 1)
@@ -135,6 +152,30 @@ __device__ __forceinline__ int tile_n(const Item& x, int j) {
 }
 // keys of sub-tile h (0: columns 0..127, 1: columns 128..) of a tile of width n
 __device__ __forceinline__ int sub_n(int n, int h) { return h == 0 ? min(n, 128) : max(0, n - 128); }
+
+// P.V order of one tile, walked by both the V producer and the MMA issuer:
+// step s of 2 * nkt (nkt = 64-key chunks of both sub-tiles, nk0 of them in
+// sub-tile 0) -> value half dh, sub-tile h, chunk kc.  An item's first tile
+// runs value half major (the previous item's epilogue hands O back one half
+// at a time); later tiles run sub-tile major (P buffer h is free as soon as
+// both value halves have used it).
+struct PvStep {
+  int dh, h, kc;
+};
+__device__ __forceinline__ PvStep pv_step(int s, int nk0, int nkt, bool first_tile) {
+  PvStep r;
+  int q;
+  if (first_tile) {
+    r.dh = s >= nkt ? 1 : 0;
+    q = s - r.dh * nkt;
+  } else {
+    r.dh = s & 1;
+    q = s >> 1;
+  }
+  r.h = q >= nk0 ? 1 : 0;
+  r.kc = q - r.h * nk0;
+  return r;
+}
 
 // 4-D tensor-map TMA copies
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
@@ -183,14 +224,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(bar(SFREE + 0), 8);
     mbar_init(bar(SFREE + 1), 8);
     mbar_init(bar(STATSFREE), 8);
-    mbar_init(bar(PFULL + 0), 4);
-    mbar_init(bar(PFULL + 1), 4);
-    mbar_init(bar(CORR), 8);
-    mbar_init(bar(OFREE), 8);
+    for (int q = 0; q < 4; ++q) mbar_init(bar(PREADY + q), 4);
+    mbar_init(bar(CORR + 0), 8);
+    mbar_init(bar(CORR + 1), 8);
+    mbar_init(bar(OFREE + 0), 8);
+    mbar_init(bar(OFREE + 1), 8);
     mbar_init(bar(STATSFULL), 4);
-    mbar_init(bar(STAGED + 0), 128);
-    mbar_init(bar(STAGED + 1), 128);
-    for (int q = 0; q < 4; ++q) mbar_init(bar(XMAX + q), 2);
+    for (int e = 0; e < 4; ++e) mbar_init(bar(STAGED + e), 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -236,8 +276,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               if (!ok) break;
               const uint32_t dst = sb + S_KRING + st * kKStage;
               if (comp) {
-                mbar_expect_tx(bar(KFULL + st), kKT * 128);
-                tma_load_3d(dst, &maps.ck, bar(KFULL + st), 64 * d, j * kKT, x.b);
+                const int n64 = (tile_n(x, j) + 63) >> 6;   // 64-row boxes this tile uses
+                mbar_expect_tx(bar(KFULL + st), n64 * 8192);
+                for (int r = 0; r < n64; ++r)
+                  tma_load_3d(dst + r * 8192, &maps.ck, bar(KFULL + st), 64 * d, j * kKT + 64 * r,
+                              x.b);
               } else {
                 mbar_expect_tx(bar(KFULL + st), kWinN * 128);
                 tma_load_3d(dst, &maps.kwin, bar(KFULL + st), 64 * d, x.t0 - 127, x.b);
@@ -285,6 +328,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         umma_commit(bar(DRAIN));
         mbar_wait(bar(DRAIN), 0, abort_flag, kWaitLimitNs, 123);
       }
+    } else if (warp >= 11) {
+      // the P copier and out store roles exist on rank 1 only
     } else {
       // --------------------------------------------------------- softmax
       const int wq = warp & 3;
@@ -293,25 +338,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int pos = row >> 6;
       const uint32_t tl = tmem + (static_cast<uint32_t>(wq * 32) << 16);
       float* xmax = reinterpret_cast<float*>(smem + S_XMAX);
-      const uint32_t peerP = mapa_shared(sb + O_P + half * kPBuf, 1);
+      volatile int* xok = reinterpret_cast<volatile int*>(smem + S_XOK);
+      uint8_t* const pscr = p.pscratch + static_cast<size_t>(pair) * kScratchPerPair;
       const uint32_t peerAlpha = mapa_shared(sb + O_ALPHA, 1);
       const uint32_t peerFlags = mapa_shared(sb + O_FLAGS, 1);
       const uint32_t peerInvl = mapa_shared(sb + O_INVL, 1);
-      const uint32_t peerPFull = mapa_shared(bar(PFULL + half), 1);
+      const uint32_t peerPReady = mapa_shared(bar(PREADY), 1);
       const uint32_t peerStatsFull = mapa_shared(bar(STATSFULL), 1);
       uint32_t sj = 0, nitem = 0, nx = 0;
-      bool ok = true;
-      for (int it = pair; it < p.items && ok; it += npairs, ++nitem) {
+      bool ok = true, both = true;
+      // A row is shared with warp (warp ^ 4's partner): both write, a 64-thread
+      // named barrier, both read.  The ok flags travel with the value, so the
+      // two warps always leave their loops at the same exchange and never
+      // wait at the named barrier for a warp that has gone.
+      auto exchange = [&](float v) -> float {
+        const uint32_t xp = nx & 1;
+        xmax[(xp * 2 + half) * 128 + row] = v;
+        if (lane == 0) xok[(xp * 2 + half) * 4 + wq] = ok ? 1 : 0;
+        named_bar_sync(1 + wq, 64);
+        const float o = xmax[(xp * 2 + (half ^ 1)) * 128 + row];
+        both = ok && xok[(xp * 2 + (half ^ 1)) * 4 + wq] != 0;
+        ++nx;
+        return o;
+      };
+      // The P stores of a tile are published one step later (after the next
+      // tile's row max), so the wait for them to drain overlaps that work.
+      uint32_t pend = 0;   // scratch slot + 1 of the unpublished sub-tile
+      auto publish = [&]() {
+        fence_proxy_async_all();  // the scratch is read by the peer's bulk copy (async proxy)
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(peerPReady + 8 * (pend - 1));
+        pend = 0;
+      };
+      for (int it = pair; it < p.items; it += npairs, ++nitem) {
         const Item x = decode_item(p, it);
         const int t = x.t0 + pos;
         const int ncp = pos ? x.nc1 : x.nc0;
         float m = -INFINITY, l = 0.f;
         for (int j = 0; j < x.ntiles; ++j, ++sj) {
           const uint32_t buf = sj & 1;
-          if (!mbar_wait_warp(bar(SFULL + buf), (sj >> 1) & 1, abort_flag, kWaitLimitNs, 130)) {
-            ok = false;
-            break;
-          }
+          if (ok) ok = mbar_wait_warp(bar(SFULL + buf), (sj >> 1) & 1, abort_flag, kWaitLimitNs, 130);
           tc_fence_after();
           const int n = tile_n(x, j);
           const int nh = sub_n(n, half);
@@ -324,38 +390,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             chi = 128 + pos;
           }
           const int c0 = 128 * half;
-          const bool full = (clo <= c0) && (chi >= c0 + 128);
           const uint32_t sbase = tl + 256 * buf + c0;
+          // One code path for full and partly masked chunks (the unrolled
+          // loops are the hot code; a second copy of each costs more in
+          // instruction fetch than the two compares per score save).
           // pass A: this half's row max of the raw scores
           float mraw = -INFINITY;
-          for (int cc = 0; cc < nh; cc += 64) {
-            uint32_t r[64];
+          // 32-column chunks keep the unrolled bodies small (instruction fetch)
+#pragma unroll 1
+          for (int cc = 0; ok && cc < nh; cc += 32) {
+            uint32_t r[32];
             tmem_ld32(sbase + cc, r);
-            tmem_ld32(sbase + cc + 32, r + 32);
             tmem_wait_ld_dep32(r);
-            reg_dep32(r + 32);
-            if (full) {
+            const int lo = clo - c0 - cc, hi = chi - c0 - cc;   // visible range in this chunk
 #pragma unroll
-              for (int c = 0; c < 64; ++c) mraw = fmaxf(mraw, __uint_as_float(r[c]));
-            } else {
-#pragma unroll
-              for (int c = 0; c < 64; ++c) {
-                const int col = c0 + cc + c;
-                if (col >= clo && col < chi) mraw = fmaxf(mraw, __uint_as_float(r[c]));
-              }
-            }
+            for (int c = 0; c < 32; ++c)
+              mraw = fmaxf(mraw, (c >= lo && c < hi) ? __uint_as_float(r[c]) : -INFINITY);
           }
-          // exchange with the warp that holds the other half of the row
-          const uint32_t xp = nx & 1;
-          xmax[(xp * 2 + half) * 128 + row] = mraw;
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(XMAX + wq));
-          if (!mbar_wait_warp(bar(XMAX + wq), nx & 1, abort_flag, kWaitLimitNs, 133)) {
-            ok = false;
-            break;
-          }
-          mraw = fmaxf(mraw, xmax[(xp * 2 + (half ^ 1)) * 128 + row]);
-          ++nx;
+          mraw = fmaxf(mraw, exchange(mraw));
+          if (!both) break;
+          if (pend) publish();
           const float mt = mraw * p.scale_log2;  // scale > 0
           float alpha = 1.f;
           bool resc = false;
@@ -365,75 +419,66 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             m = mt;
           }
           const float mu = (m == -INFINITY) ? 0.f : m;
-          // the O-CTA has finished reading this half's P buffer (previous tile)
-          if (!mbar_wait_cluster_warp(bar(PFREE + half), (sj & 1) ^ 1, abort_flag, kWaitLimitNs,
-                                      131)) {
-            ok = false;
-            break;
-          }
-          // pass B: probabilities, written straight into the O-CTA's P buffer
+          // scratch slot of this (tile parity, half): free once the O-CTA has
+          // finished P.V of the tile two back
+          const uint32_t slot = (sj & 1) * 2 + half;
+          if (ok)
+            ok = mbar_wait_cluster_warp(bar(PFREE + slot), ((sj >> 1) & 1) ^ 1, abort_flag,
+                                        kWaitLimitNs, 131);
+          uint8_t* const gdst = pscr + slot * 32768;
+          // pass B: probabilities into the scratch slot
           float rs = 0.f;
-          for (int cc = 0; cc < nh; cc += 64) {
-            uint32_t r[64];
+#pragma unroll 1
+          for (int cc = 0; ok && cc < nh; cc += 32) {
+            uint32_t r[32];
             tmem_ld32(sbase + cc, r);
-            tmem_ld32(sbase + cc + 32, r + 32);
             tmem_wait_ld_dep32(r);
-            reg_dep32(r + 32);
-            uint32_t pk[32];
+            uint32_t pk[16];
+            const int lo = clo - c0 - cc, hi = chi - c0 - cc;
 #pragma unroll
-            for (int c = 0; c < 64; c += 2) {
-              const int col = c0 + cc + c;
-              float e0 = ex2_approx(fmaf(__uint_as_float(r[c]), p.scale_log2, -mu));
-              float e1 = ex2_approx(fmaf(__uint_as_float(r[c + 1]), p.scale_log2, -mu));
-              if (!full) {
-                e0 = (col >= clo && col < chi) ? e0 : 0.f;
-                e1 = (col + 1 >= clo && col + 1 < chi) ? e1 : 0.f;
-              }
+            for (int c = 0; c < 32; c += 2) {
+              // masked scores enter ex2 as -inf and come out as 0
+              const float x0 = (c >= lo && c < hi) ? fmaf(__uint_as_float(r[c]), p.scale_log2, -mu)
+                                                   : -INFINITY;
+              const float x1 = (c + 1 >= lo && c + 1 < hi)
+                                   ? fmaf(__uint_as_float(r[c + 1]), p.scale_log2, -mu)
+                                   : -INFINITY;
+              const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
               rs += e0 + e1;
               pk[c / 2] = pack_bf16x2(e0, e1);
             }
+            // chunk-major image: 8-key chunk k8 of row `row` at k8 * 2048 + 16 * row,
+            // so the 32 lanes of a warp store 512 contiguous bytes
 #pragma unroll
-            for (int c8 = 0; c8 < 8; ++c8) {
-              const int k8 = (cc >> 3) + c8;   // 8-key chunk index within the sub-tile
-              const uint32_t off = (k8 >> 3) * 16384 + sw128_offset(row, k8 & 7);
-              st_cluster_v4(peerP + off, pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2],
-                            pk[4 * c8 + 3]);
+            for (int c8 = 0; c8 < 4; ++c8) {
+              const int k8 = (cc >> 3) + c8;
+              *reinterpret_cast<uint4*>(gdst + k8 * 2048 + 16 * row) =
+                  make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
             }
           }
-          if (half == 0) {
-            st_cluster_b32(peerAlpha + 4 * row, __float_as_uint(alpha));
+          if (ok && half == 0) {
+            st_cluster_b32(peerAlpha + 512 * (sj & 1) + 4 * row, __float_as_uint(alpha));
             const int any = __any_sync(0xffffffffu, resc) ? 1 : 0;
-            if (lane == 0) st_cluster_b32(peerFlags + 4 * wq, static_cast<uint32_t>(any));
+            if (lane == 0)
+              st_cluster_b32(peerFlags + 16 * (sj & 1) + 4 * wq, static_cast<uint32_t>(any));
           }
-          fence_proxy_async_all();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) {
-            mbar_arrive_cluster(peerPFull);
-            mbar_arrive(bar(SFREE + buf));
-          }
+          if (lane == 0) mbar_arrive(bar(SFREE + buf));  // S buffer read out
+          pend = slot + 1;
           l = l * alpha + rs;
         }
-        if (!ok) break;
-        // row sum = both halves (one more round of the same exchange); 1/l to
-        // the O-CTA epilogue, lse to the caller
-        {
-          const uint32_t xp = nx & 1;
-          xmax[(xp * 2 + half) * 128 + row] = l;
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(XMAX + wq));
-          if (!mbar_wait_warp(bar(XMAX + wq), nx & 1, abort_flag, kWaitLimitNs, 134)) {
-            ok = false;
-            break;
-          }
-          l += xmax[(xp * 2 + (half ^ 1)) * 128 + row];
-          ++nx;
-        }
+        if (!both) break;
+        // row sum = both halves (one more exchange); 1/l to the O-CTA
+        // epilogue, lse to the caller
+        l += exchange(l);
+        if (!both) break;
+        if (pend) publish();
         if (half == 0) {
           if (!mbar_wait_cluster_warp(bar(STATSFREE), (nitem & 1) ^ 1, abort_flag, kWaitLimitNs,
                                       132)) {
             ok = false;
-            break;
+            continue;  // the next exchange takes both warps out
           }
           st_cluster_b32(peerInvl + 4 * row, __float_as_uint(1.f / l));
           __syncwarp();
@@ -448,6 +493,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // =====================================================================
     // O-CTA
     // =====================================================================
+    // V stage uses of one item: per tile, both value halves of every 64-key
+    // chunk of both sub-tiles
+    auto v_uses = [&](const Item& x) -> uint32_t {
+      uint32_t n_uses = 0;
+      for (int j = 0; j < x.ntiles; ++j) {
+        const int n = tile_n(x, j);
+        n_uses += 2 * ((sub_n(n, 0) + 63) / 64) + 2 * ((sub_n(n, 1) + 63) / 64);
+      }
+      return n_uses;
+    };
     if (warp <= 1) {
       // --------------------------------------------------------- producers
       if (lane == 0) {
@@ -471,63 +526,137 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int j = 0; j < x.ntiles && ok; ++j) {
             const int n = tile_n(x, j);
             const bool comp = j < x.n_ctiles;
-            for (int h = 0; h < 2 && ok; ++h) {
-              const int nh = sub_n(n, h);
-              for (int kc = 0; kc * 64 < nh && ok; ++kc) {
-                for (int dh = 0; dh < 2 && ok; ++dh) {
-                  if (comp) ok = stage_load(&maps.cv4, j * kKT + 128 * h + 64 * kc, 4 * dh, x.b);
-                  else ok = stage_load(&maps.v4, x.t0 - 127 + 128 * h + 64 * kc, 4 * dh, x.b);
-                }
-              }
+            const int nk0 = (sub_n(n, 0) + 63) >> 6;
+            const int nkt = nk0 + ((sub_n(n, 1) + 63) >> 6);
+            for (int s = 0; s < 2 * nkt && ok; ++s) {
+              const PvStep q = pv_step(s, nk0, nkt, j == 0);
+              const int key = 128 * q.h + 64 * q.kc;
+              ok = stage_load(comp ? &maps.cv4 : &maps.v4, comp ? j * kKT + key : x.t0 - 127 + key,
+                              4 * q.dh, x.b);
             }
           }
           for (int e = 0; e < 4 && ok; ++e) ok = stage_load(&maps.g4, x.t0 * kHeads, 2 * e, x.b);
         }
       }
+    } else if (warp == 11) {
+      // --------------------------------------------------------- P copier
+      if (lane == 0) {
+        const uint8_t* const pscr = p.pscratch + static_cast<size_t>(pair) * kScratchPerPair;
+        uint32_t sj = 0;
+        bool ok = true;
+        for (int it = pair; it < p.items && ok; it += npairs) {
+          const Item x = decode_item(p, it);
+          for (int j = 0; j < x.ntiles && ok; ++j, ++sj) {
+            const int n = tile_n(x, j);
+            for (int h = 0; h < 2 && ok; ++h) {
+              const int nh = sub_n(n, h);
+              ok = mbar_wait_cluster(bar(PREADY + (sj & 1) * 2 + h), (sj >> 1) & 1, abort_flag,
+                                     kWaitLimitNs, 145) &&
+                   mbar_wait(bar(PBUFFREE + h), (sj & 1) ^ 1, abort_flag, kWaitLimitNs, 146);
+              if (!ok) break;
+              if (nh > 0) {
+                fence_proxy_async_all();
+                const uint32_t bytes = nh > 64 ? 32768u : 16384u;
+                mbar_expect_tx(bar(PFULL + h), bytes);
+                asm volatile(
+                    "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes"
+                    " [%0], [%1], %2, [%3];" ::"r"(sb + O_P + h * kPBuf),
+                    "l"(pscr + ((sj & 1) * 2 + h) * 32768), "r"(bytes), "r"(bar(PFULL + h))
+                    : "memory");
+              } else {
+                mbar_arrive(bar(PFULL + h));
+              }
+            }
+          }
+        }
+      }
+    } else if (warp == 12) {
+      // --------------------------------------------------------- out stores
+      // The epilogue writes out over the g image of each 128-column stage;
+      // this warp stores the stage and hands it back to the producers once
+      // the copy engine has read it.
+      if (lane == 0) {
+        uint32_t ubase = 0, nitem = 0;
+        bool ok = true;
+        for (int it = pair; it < p.items && ok; it += npairs, ++nitem) {
+          const Item x = decode_item(p, it);
+          const uint32_t gbase = ubase + v_uses(x);
+          ubase = gbase + 4;
+          for (int e = 0; e < 4 && ok; ++e) {
+            const uint32_t st = (gbase + e) % kVStages;
+            ok = mbar_wait(bar(STAGED + e), nitem & 1, abort_flag, kWaitLimitNs, 170);
+            if (!ok) break;
+            tma_store_4d(&maps.out4, sb + O_VRING + st * kVStage, 0, x.t0 * kHeads, 2 * e, x.b);
+            bulk_commit();
+            if (e & 1) {
+              // both stages of this value half are in flight: release them as
+              // their reads complete
+              bulk_wait_read_n<1>();
+              mbar_arrive(bar(VEMPTY + (gbase + e - 1) % kVStages));
+              bulk_wait_read_all();
+              mbar_arrive(bar(VEMPTY + st));
+            }
+          }
+        }
+        bulk_wait_all();
+      }
     } else if (warp == 2) {
       // --------------------------------------------------------- MMA (O += P V)
       if (lane == 0) {
-        uint32_t u = 0, sj = 0, nitem = 0;
+        uint32_t u = 0, sj = 0, nitem = 0, ncorr = 0;
         bool ok = true;
         const uint32_t idesc = idesc_bf16_f32(kRows, 256, false, true);
         for (int it = pair; it < p.items && ok; it += npairs, ++nitem) {
           const Item x = decode_item(p, it);
           for (int j = 0; j < x.ntiles && ok; ++j, ++sj) {
             const int n = tile_n(x, j);
-            for (int h = 0; h < 2 && ok; ++h) {
+            if (j > 0) {  // an item's first tile never needs a rescale of O
+              ok = mbar_wait(bar(CORR + (ncorr & 1)), (ncorr >> 1) & 1, abort_flag, kWaitLimitNs,
+                             151);
+              ++ncorr;
+            }
+            // P.V of one 64-key chunk into one value half
+            auto chunk = [&](int dh, int h, int kc) {
               const int nh = sub_n(n, h);
-              ok = mbar_wait_cluster(bar(PFULL + h), sj & 1, abort_flag, kWaitLimitNs, 150);
-              if (!ok) break;
-              if (h == 0) {
-                ok = mbar_wait(bar(CORR), sj & 1, abort_flag, kWaitLimitNs, 151);
-                if (!ok) break;
-                if (j == 0) {
-                  ok = mbar_wait(bar(OFREE), (nitem & 1) ^ 1, abort_flag, kWaitLimitNs, 152);
-                  if (!ok) break;
-                }
-              }
+              const int ksteps = min(4, (nh - 64 * kc) >> 4);
+              const uint32_t st = u % kVStages;
+              ok = mbar_wait(bar(VFULL + st), (u / kVStages) & 1, abort_flag, kWaitLimitNs, 153);
+              ++u;
+              if (!ok) return;
               tc_fence_after();
               const uint32_t pa = sb + O_P + h * kPBuf;
-              for (int kc = 0; kc * 64 < nh && ok; ++kc) {
-                const int ksteps = min(4, (nh - 64 * kc) >> 4);
-                for (int dh = 0; dh < 2; ++dh, ++u) {
-                  const uint32_t st = u % kVStages;
-                  ok = mbar_wait(bar(VFULL + st), (u / kVStages) & 1, abort_flag, kWaitLimitNs, 153);
-                  if (!ok) break;
-                  tc_fence_after();
-                  const uint32_t va = sb + O_VRING + st * kVStage;
-                  for (int ks = 0; ks < ksteps; ++ks) {
-                    const bool first = (j == 0 && h == 0 && kc == 0 && ks == 0);
-                    umma_bf16(tmem + 256 * dh, sdesc_sw128(pa + kc * 16384 + 32 * ks, 16, 1024),
-                              sdesc_sw128(va + 2048 * ks, 8192, 1024), idesc, first ? 0u : 1u);
-                  }
-                  umma_commit(bar(VEMPTY + st));
-                }
+              const uint32_t va = sb + O_VRING + st * kVStage;
+              for (int ks = 0; ks < ksteps; ++ks) {
+                const bool first = (j == 0 && h == 0 && kc == 0 && ks == 0);
+                umma_bf16(tmem + 256 * dh, sdesc_noswz(pa + kc * 16384 + 4096 * ks, 2048, 128),
+                          sdesc_sw128(va + 2048 * ks, 8192, 1024), idesc, first ? 0u : 1u);
               }
-              if (!ok) break;
-              umma_commit(bar(PVDONE));
-              umma_commit_mc(bar(PFREE + h), 0x1);  // sub-tile buffer h is free again (rank 0)
+              umma_commit(bar(VEMPTY + st));
+            };
+            auto p_full = [&](int h) {
+              if (ok) ok = mbar_wait(bar(PFULL + h), sj & 1, abort_flag, kWaitLimitNs, 150);
+              tc_fence_after();
+            };
+            auto p_done = [&](int h) {
+              umma_commit(bar(PBUFFREE + h));                       // smem P buffer h reusable
+              umma_commit_mc(bar(PFREE + (sj & 1) * 2 + h), 0x1);   // scratch slot reusable (rank 0)
+            };
+            const int nk0 = (sub_n(n, 0) + 63) >> 6, nk1 = (sub_n(n, 1) + 63) >> 6;
+            const int nkt = nk0 + nk1;
+            for (int s = 0; s < 2 * nkt && ok; ++s) {
+              const PvStep q = pv_step(s, nk0, nkt, j == 0);
+              if (j == 0 && (s == 0 || s == nkt))  // this half of the last item's O is read out
+                ok = mbar_wait(bar(OFREE + q.dh), (nitem & 1) ^ 1, abort_flag, kWaitLimitNs, 152);
+              if (q.dh == 0 && q.kc == 0) p_full(q.h);
+              if (ok) chunk(q.dh, q.h, q.kc);
+              if (ok && q.dh == 1 && q.kc == (q.h ? nk1 : nk0) - 1) p_done(q.h);
             }
+            if (ok && nk1 == 0) {  // empty sub-tile 1: its buffer handshake still runs
+              p_full(1);
+              if (ok) p_done(1);
+            }
+            if (!ok) break;
+            umma_commit(bar(PVDONE + (sj & 1)));   // all of tile sj's P.V
           }
           if (!ok) break;
           umma_commit(bar(OFULL));
@@ -539,35 +668,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     } else {
       // --------------------------------------------------------- correction + epilogue
       const int wq = warp & 3;
-      const int half = (warp - 3) >> 2;       // value columns [256 half, 256 half + 256)
+      const int half = (warp - 3) >> 2;
       const int row = wq * 32 + lane;
-      const uint32_t tl = tmem + (static_cast<uint32_t>(wq * 32) << 16) + 256 * half;
+      const uint32_t tq = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+      const uint32_t tl = tq + 256 * half;     // rescale: value columns [256 half, +256)
       const volatile int* flags = reinterpret_cast<const volatile int*>(smem + O_FLAGS);
       const volatile float* alpha_s = reinterpret_cast<const volatile float*>(smem + O_ALPHA);
       const volatile float* invl_s = reinterpret_cast<const volatile float*>(smem + O_INVL);
       const uint32_t peerStatsFree = mapa_shared(bar(STATSFREE), 0);
-      uint32_t sj = 0, nitem = 0, pv = 0, ubase = 0;
+      uint32_t sj = 0, nitem = 0, ubase = 0, ncorr = 0;
       bool ok = true;
       for (int it = pair; it < p.items && ok; it += npairs, ++nitem) {
         const Item x = decode_item(p, it);
-        uint32_t vstages = 0;
-        for (int j = 0; j < x.ntiles; ++j, ++sj) {
-          const int n = tile_n(x, j);
-          vstages += 2 * ((sub_n(n, 0) + 63) / 64) + 2 * ((sub_n(n, 1) + 63) / 64);
-          if (!mbar_wait_cluster_warp(bar(PFULL), sj & 1, abort_flag, kWaitLimitNs, 160)) {
+        ++sj;  // the first tile of an item needs no correction (its running max starts there)
+        for (int j = 1; j < x.ntiles; ++j, ++sj, ++ncorr) {
+          if (!mbar_wait_cluster_warp(bar(PREADY + (sj & 1) * 2), (sj >> 1) & 1, abort_flag,
+                                      kWaitLimitNs, 160)) {
             ok = false;
             break;
           }
           // rarely: rescale O rows before the next P.V accumulates into them
-          const bool any = (flags[0] | flags[1] | flags[2] | flags[3]) != 0;
+          const volatile int* fl = flags + 4 * (sj & 1);
+          const bool any = (fl[0] | fl[1] | fl[2] | fl[3]) != 0;
           if (any) {
-            // wait for every P.V issued so far (the last one is sub-tile 1 of tile j-1)
-            if (!mbar_wait_warp(bar(PVDONE), (pv + 1) & 1, abort_flag, kWaitLimitNs, 161)) {
+            // wait for every P.V of the previous tile
+            const uint32_t pj = sj - 1;
+            if (!mbar_wait_warp(bar(PVDONE + (pj & 1)), (pj >> 1) & 1, abort_flag, kWaitLimitNs,
+                                161)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const float a = alpha_s[row];
+            const float a = alpha_s[128 * (sj & 1) + row];
             uint32_t r[32];
 #pragma unroll 1
             for (int c = 0; c < 256; c += 32) {
@@ -581,8 +713,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar(CORR));
-          pv += 2;  // P.V of both sub-tiles of this tile will be committed to PVDONE
+          if (lane == 0) mbar_arrive(bar(CORR + (ncorr & 1)));
         }
         if (!ok) break;
         // ---------------------------------------------------------- epilogue
@@ -595,10 +726,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const float il = invl_s[row];
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(peerStatsFree);
-        const uint32_t gbase = ubase + vstages;
+        const uint32_t gbase = ubase + v_uses(x);
         ubase = gbase + 4;
+        // value half ee first (both warps of a quadrant, 128 columns each), so
+        // O half 0 is released to the next item halfway through
         for (int ee = 0; ee < 2; ++ee) {
-          const int e = 2 * half + ee;          // g / out stage: value columns [128e, 128e + 128)
+          const int e = half + 2 * ee;          // g / out stage: value columns [128e, 128e + 128)
           const uint32_t ug = gbase + e;
           const uint32_t st = ug % kVStages;
           if (!mbar_wait_warp(bar(VFULL + st), (ug / kVStages) & 1, abort_flag, kWaitLimitNs, 164)) {
@@ -606,27 +739,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             break;
           }
           uint8_t* stage = smem + O_VRING + st * kVStage;
+          // 32 value columns per step: a 64-column slab of the stage holds
+          // steps 2 sl and 2 sl + 1
 #pragma unroll 1
-          for (int sl = 0; sl < 2; ++sl) {
-            uint32_t o[64];
-            tmem_ld32(tl + 128 * ee + 64 * sl, o);
-            tmem_ld32(tl + 128 * ee + 64 * sl + 32, o + 32);
+          for (int q32 = 0; q32 < 4; ++q32) {
+            const int sl = q32 >> 1;
+            uint32_t o[32];
+            tmem_ld32(tq + 128 * e + 32 * q32, o);
             tmem_wait_ld_dep32(o);
-            reg_dep32(o + 32);
-            if (ee == 1 && sl == 1) {
+            if (q32 == 3) {
               tc_fence_before();
               __syncwarp();
-              if (lane == 0) mbar_arrive(bar(OFREE));
+              if (lane == 0) mbar_arrive(bar(OFREE + ee));
             }
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
+            for (int c4 = 0; c4 < 4; ++c4) {
+              const int c = 4 * (q32 & 1) + c4;   // 16-byte chunk of the 128-byte slab row
               uint4* ptr = reinterpret_cast<uint4*>(stage + sl * 16384 + sw128_offset(row, c));
               const uint4 gv = *ptr;
               const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
               uint32_t ow[4];
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
-                const int oc = 8 * c + 2 * q;
+                const int oc = 8 * c4 + 2 * q;
                 ow[q] = pack_bf16x2(__uint_as_float(o[oc]) * il * sigmoid_fast(bf16lo_to_f32(gw[q])),
                                     __uint_as_float(o[oc + 1]) * il *
                                         sigmoid_fast(bf16hi_to_f32(gw[q])));
@@ -635,19 +770,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
           }
           fence_proxy_async_smem();
-          mbar_arrive(bar(STAGED + half));
-          if (warp == 3 + 4 * half && lane == 0) {
-            if (mbar_wait(bar(STAGED + half), (2u * nitem + ee) & 1, abort_flag, kWaitLimitNs,
-                          165)) {
-              tma_store_4d(&maps.out4, sb + O_VRING + st * kVStage, 0, x.t0 * kHeads, 2 * e, x.b);
-              bulk_commit();
-              bulk_wait_read_all();
-              mbar_arrive(bar(VEMPTY + st));
-            }
-          }
+          mbar_arrive(bar(STAGED + e));
         }
       }
-      if (lane == 0 && (warp == 3 || warp == 7)) bulk_wait_all();
     }
   }
 

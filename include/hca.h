@@ -73,6 +73,13 @@ hca_status_t hca_compress(const hca_bf16* k, const hca_bf16* v, const hca_bf16* 
                           hca_bf16* ck, hca_bf16* cv, hca_stream_t stream);
 
 /*
+ * hca_prefill_workspace_size — bytes of device scratch hca_prefill_fwd needs
+ * on the current device (probability tiles in flight between the two CTAs of
+ * each cluster; about 128 KB per cluster, under 10 MB on a B200).
+ */
+size_t hca_prefill_workspace_size(int B, int T);
+
+/*
  * hca_prefill_fwd — HCA attention for every position of B sequences.
  *   For query t of batch b and head h (page sources as above):
  *     keys   = [ck[b, 0 : nc(t)] ; k[b, max(0, t-127) : t+1]]
@@ -82,15 +89,19 @@ hca_status_t hca_compress(const hca_bf16* k, const hca_bf16* v, const hca_bf16* 
  *   lse (optional) receives ln(sum exp(scale * keys . q)) per (b, t, h).
  * Layout:  q, g, out [B, T, H, 512] bf16 (H = 64);  k, v [B, T, 512] bf16;
  *          ck, cv [B, floor(T/128), 512] bf16 as written by hca_compress;
- *          lse [B, T, H] fp32 or NULL.
+ *          lse [B, T, H] fp32 or NULL;  ws: caller-owned device scratch of at
+ *          least hca_prefill_workspace_size(B, T) bytes, 256-byte aligned (its
+ *          contents need no initialisation and are meaningless afterwards;
+ *          two calls in flight at once need two workspaces).
  * Errors:  H != 64 -> HCA_ERR_UNSUPPORTED; B < 1, T < 1, a null pointer (other
- *          than lse), a pointer not 16-byte aligned, or a non-finite or
- *          non-positive scale -> HCA_ERR_INVALID_ARG.
+ *          than lse), a pointer not 16-byte aligned, a workspace too small or
+ *          misaligned, or a non-finite or non-positive scale ->
+ *          HCA_ERR_INVALID_ARG.
  */
 hca_status_t hca_prefill_fwd(const hca_bf16* q, const hca_bf16* k, const hca_bf16* v,
                              const hca_bf16* ck, const hca_bf16* cv, const hca_bf16* g, int B,
-                             int T, int H, float scale, hca_bf16* out, float* lse,
-                             hca_stream_t stream);
+                             int T, int H, float scale, hca_bf16* out, float* lse, void* ws,
+                             size_t ws_bytes, hca_stream_t stream);
 
 /*
  * hca_decode_workspace_size — bytes of scratch hca_decode needs for S

@@ -60,13 +60,15 @@ def test_compress_rejects_bad_args(lib):
 
 def test_prefill_rejects_bad_args(lib):
     vp, i = ctypes.c_void_p, ctypes.c_int
-    lib.hca_prefill_fwd.argtypes = [vp] * 6 + [i, i, i, ctypes.c_float, vp, vp, vp]
+    lib.hca_prefill_fwd.argtypes = [vp] * 6 + [i, i, i, ctypes.c_float, vp, vp, vp,
+                                                ctypes.c_size_t, vp]
     f = 0x10000
-    ok_args = [f, f, f, f, f, f, 1, 256, 64, 0.04, f, None, None]
+    ok_args = [f, f, f, f, f, f, 1, 256, 64, 0.04, f, None, f, 1 << 30, None]
 
     def call(**kw):
         a = list(ok_args)
-        names = ["q", "k", "v", "ck", "cv", "g", "B", "T", "H", "scale", "out", "lse", "st"]
+        names = ["q", "k", "v", "ck", "cv", "g", "B", "T", "H", "scale", "out", "lse", "ws",
+                 "ws_bytes", "st"]
         for k2, v2 in kw.items():
             a[names.index(k2)] = v2
         return lib.hca_prefill_fwd(*a)
@@ -80,6 +82,8 @@ def test_prefill_rejects_bad_args(lib):
     assert call(out=None) == 1
     assert call(ck=None) == 1          # T = 256 has compressed entries
     assert call(g=f + 8) == 1          # misaligned
+    assert call(ws=None) == 1          # no workspace
+    assert call(ws=f + 16) == 1        # workspace not 256-byte aligned
 
 
 def test_decode_rejects_bad_args(lib):
