@@ -268,6 +268,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                       x.b);
           for (int j = 0; j < x.ntiles && ok; ++j) {
             const bool comp = j < x.n_ctiles;
+#pragma unroll 1
             for (int d = 0; d < 8; ++d, ++u) {
               if ((u & 1) != static_cast<uint32_t>(me)) continue;
               const uint32_t st = u % kKStages;
@@ -278,6 +279,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               if (comp) {
                 const int n64 = (tile_n(x, j) + 63) >> 6;   // 64-row boxes this tile uses
                 mbar_expect_tx(bar(KFULL + st), n64 * 8192);
+#pragma unroll 1
                 for (int r = 0; r < n64; ++r)
                   tma_load_3d(dst + r * 8192, &maps.ck, bar(KFULL + st), 64 * d, j * kKT + 64 * r,
                               x.b);
@@ -303,6 +305,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const uint32_t idesc = idesc_bf16_f32(kRows, tile_n(x, j), false, false);
             const uint32_t dS = tmem + 256 * buf;
+#pragma unroll 1
             for (int d = 0; d < 8 && ok; ++d, ++u) {
               if (j == 0 && (d & 3) == 0) {
                 ok = mbar_wait(bar(QFULL + (d >> 2)), nitem & 1, abort_flag, kWaitLimitNs, 121);
@@ -523,6 +526,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         };
         for (int it = pair; it < p.items && ok; it += npairs) {
           const Item x = decode_item(p, it);
+          if (me == 0) {  // warm L2 with this item's gate rows; they are staged after its V
+#pragma unroll 1
+            for (int e = 0; e < 4; ++e) tma_prefetch_4d(&maps.g4, 0, x.t0 * kHeads, 2 * e, x.b);
+          }
           for (int j = 0; j < x.ntiles && ok; ++j) {
             const int n = tile_n(x, j);
             const bool comp = j < x.n_ctiles;
@@ -535,6 +542,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                               4 * q.dh, x.b);
             }
           }
+#pragma unroll 1
           for (int e = 0; e < 4 && ok; ++e) ok = stage_load(&maps.g4, x.t0 * kHeads, 2 * e, x.b);
         }
       }
@@ -548,6 +556,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const Item x = decode_item(p, it);
           for (int j = 0; j < x.ntiles && ok; ++j, ++sj) {
             const int n = tile_n(x, j);
+#pragma unroll 1
             for (int h = 0; h < 2 && ok; ++h) {
               const int nh = sub_n(n, h);
               ok = mbar_wait_cluster(bar(PREADY + (sj & 1) * 2 + h), (sj >> 1) & 1, abort_flag,
@@ -582,6 +591,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const Item x = decode_item(p, it);
           const uint32_t gbase = ubase + v_uses(x);
           ubase = gbase + 4;
+#pragma unroll 1
           for (int e = 0; e < 4 && ok; ++e) {
             const uint32_t st = (gbase + e) % kVStages;
             ok = mbar_wait(bar(STAGED + e), nitem & 1, abort_flag, kWaitLimitNs, 170);
@@ -626,6 +636,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               tc_fence_after();
               const uint32_t pa = sb + O_P + h * kPBuf;
               const uint32_t va = sb + O_VRING + st * kVStage;
+#pragma unroll 1
               for (int ks = 0; ks < ksteps; ++ks) {
                 const bool first = (j == 0 && h == 0 && kc == 0 && ks == 0);
                 umma_bf16(tmem + 256 * dh, sdesc_noswz(pa + kc * 16384 + 4096 * ks, 2048, 128),
@@ -730,6 +741,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         ubase = gbase + 4;
         // value half ee first (both warps of a quadrant, 128 columns each), so
         // O half 0 is released to the next item halfway through
+#pragma unroll 1
         for (int ee = 0; ee < 2; ++ee) {
           const int e = half + 2 * ee;          // g / out stage: value columns [128e, 128e + 128)
           const uint32_t ug = gbase + e;
