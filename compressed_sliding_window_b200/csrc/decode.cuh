@@ -589,6 +589,10 @@ __global__ void __launch_bounds__(32 * kCombineHeads)
   };
   const int c0 = owner(P0), c1 = owner(P1 - 1);
   const int np = c1 - c0 + 1;
+  // the gate row is independent of the partials: start its load first
+  const size_t obase = (static_cast<size_t>(s) * kHeads + h) * kDim + 16 * lane;
+  const uint4* gp = reinterpret_cast<const uint4*>(g + obase);
+  const uint4 gv0 = __ldg(gp), gv1 = __ldg(gp + 1);
   auto nonempty = [&](int c) { return N * c / grid < N * (c + 1) / grid; };
   // pass 1: M = max of the partial maxima
   float M = -INFINITY;
@@ -615,31 +619,47 @@ __global__ void __launch_bounds__(32 * kCombineHeads)
     }
     L += lw;
     const int cnt = min(32, np - base);
-    for (int i = 0; i < cnt; ++i) {
-      const float wi = __shfl_sync(0xffffffffu, w, i);
-      if (wi == 0.f) continue;  // empty split (or a fully masked one)
-      const size_t slot = static_cast<size_t>(c0 + base + i + s);
-      const float4* src = reinterpret_cast<const float4*>(p.ws_o + (slot * kHeads + h) * kDim) +
-                          lane * 4;
+    // four partial rows per round, all of their loads issued before any use
+#pragma unroll 1
+    for (int i0 = 0; i0 < cnt; i0 += 4) {
+      float wv[4];
+      float4 o[4][4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float4 o = __ldg(src + q);
-        acc[4 * q + 0] = fmaf(wi, o.x, acc[4 * q + 0]);
-        acc[4 * q + 1] = fmaf(wi, o.y, acc[4 * q + 1]);
-        acc[4 * q + 2] = fmaf(wi, o.z, acc[4 * q + 2]);
-        acc[4 * q + 3] = fmaf(wi, o.w, acc[4 * q + 3]);
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u;
+        wv[u] = __shfl_sync(0xffffffffu, w, i & 31);
+        // skipped: past the last partial, an empty split, or a fully masked one
+        if (i >= cnt || wv[u] == 0.f) {
+          wv[u] = 0.f;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) o[u][q] = make_float4(0.f, 0.f, 0.f, 0.f);
+        } else {
+          const size_t slot = static_cast<size_t>(c0 + base + i + s);
+          const float4* src =
+              reinterpret_cast<const float4*>(p.ws_o + (slot * kHeads + h) * kDim) + lane * 4;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) o[u][q] = __ldg(src + q);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          acc[4 * q + 0] = fmaf(wv[u], o[u][q].x, acc[4 * q + 0]);
+          acc[4 * q + 1] = fmaf(wv[u], o[u][q].y, acc[4 * q + 1]);
+          acc[4 * q + 2] = fmaf(wv[u], o[u][q].z, acc[4 * q + 2]);
+          acc[4 * q + 3] = fmaf(wv[u], o[u][q].w, acc[4 * q + 3]);
+        }
       }
     }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
   const float inv = 1.f / L;
-  const size_t base = (static_cast<size_t>(s) * kHeads + h) * kDim + 16 * lane;
-  const uint4* gp = reinterpret_cast<const uint4*>(g + base);
-  uint4* op = reinterpret_cast<uint4*>(out + base);
+  uint4* op = reinterpret_cast<uint4*>(out + obase);
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
-    const uint4 gv = __ldg(gp + q);
+    const uint4 gv = q ? gv1 : gv0;
     const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
     uint32_t ow[4];
 #pragma unroll
