@@ -563,9 +563,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---------------------------------------------------------------------------
 // Combine: CTA (sequence s, 8 heads), one warp per head, 16 value columns per
-// lane.  The weights 2^(m_c - M) of all partials are computed in parallel
-// across lanes and broadcast with shuffles, so the partial rows stream with
-// independent loads.
+// lane.  The partials are merged online (running max, rescaled accumulator),
+// two per round, so the loads of a round's (m, l) and its partial rows go out
+// together and the kernel needs few enough registers to run in one wave.
+// Empty splits are recognised arithmetically; a split whose keys were all
+// masked has m = -inf, weight 0 and a zero row.
 // ---------------------------------------------------------------------------
 constexpr int kCombineHeads = 8;
 
@@ -577,10 +579,14 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 __global__ void __launch_bounds__(32 * kCombineHeads)
     combine_kernel(const Params p, int grid, const uint16_t* __restrict__ g,
                    uint16_t* __restrict__ out) {
-  pdl_wait();  // the split pass (a prerequisite grid) has finished and its writes are visible
   const int s = blockIdx.x;
   const int h = blockIdx.y * kCombineHeads + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  // the gate row does not depend on the split pass: load it before waiting
+  const size_t obase = (static_cast<size_t>(s) * kHeads + h) * kDim + 16 * lane;
+  const uint4* gp = reinterpret_cast<const uint4*>(g + obase);
+  const uint4 gv0 = __ldg(gp), gv1 = __ldg(gp + 1);
+  pdl_wait();  // the split pass (a prerequisite grid) has finished and its writes are visible
   const long long N = p.seq_tile[p.S];
   const long long P0 = p.seq_tile[s], P1 = p.seq_tile[s + 1];
   // CTA that owns global tile x: ceil((x + 1) * grid / N) - 1
@@ -589,72 +595,48 @@ __global__ void __launch_bounds__(32 * kCombineHeads)
   };
   const int c0 = owner(P0), c1 = owner(P1 - 1);
   const int np = c1 - c0 + 1;
-  // the gate row is independent of the partials: start its load first
-  const size_t obase = (static_cast<size_t>(s) * kHeads + h) * kDim + 16 * lane;
-  const uint4* gp = reinterpret_cast<const uint4*>(g + obase);
-  const uint4 gv0 = __ldg(gp), gv1 = __ldg(gp + 1);
   auto nonempty = [&](int c) { return N * c / grid < N * (c + 1) / grid; };
-  // pass 1: M = max of the partial maxima
-  float M = -INFINITY;
-  for (int base = 0; base < np; base += 32) {
-    const int c = c0 + base + lane;
-    if (base + lane < np && nonempty(c))
-      M = fmaxf(M, p.ws_ml[static_cast<size_t>(c + s) * 128 + h]);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  const float Mu = (M == -INFINITY) ? 0.f : M;
-  // pass 2: weighted sum of the partial rows and of their denominators
   float acc[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-  float L = 0.f;
-  for (int base = 0; base < np; base += 32) {
-    const int c = c0 + base + lane;
-    float w = 0.f, lw = 0.f;
-    if (base + lane < np && nonempty(c)) {
-      const size_t slot = static_cast<size_t>(c + s);
-      w = ex2_approx(p.ws_ml[slot * 128 + h] - Mu);
-      lw = w * p.ws_ml[slot * 128 + 64 + h];
-    }
-    L += lw;
-    const int cnt = min(32, np - base);
-    // four partial rows per round, all of their loads issued before any use
+  float M = -INFINITY, L = 0.f;
 #pragma unroll 1
-    for (int i0 = 0; i0 < cnt; i0 += 4) {
-      float wv[4];
-      float4 o[4][4];
+  for (int i0 = 0; i0 < np; i0 += 2) {
+    float m2[2], l2[2];
+    float4 o[2][4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = i0 + u;
-        wv[u] = __shfl_sync(0xffffffffu, w, i & 31);
-        // skipped: past the last partial, an empty split, or a fully masked one
-        if (i >= cnt || wv[u] == 0.f) {
-          wv[u] = 0.f;
+    for (int u = 0; u < 2; ++u) {
+      const int c = c0 + i0 + u;
+      if (i0 + u < np && nonempty(c)) {
+        const size_t slot = static_cast<size_t>(c + s);
+        m2[u] = __ldg(p.ws_ml + slot * 128 + h);
+        l2[u] = __ldg(p.ws_ml + slot * 128 + 64 + h);
+        const float4* src =
+            reinterpret_cast<const float4*>(p.ws_o + (slot * kHeads + h) * kDim) + lane * 4;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) o[u][q] = make_float4(0.f, 0.f, 0.f, 0.f);
-        } else {
-          const size_t slot = static_cast<size_t>(c0 + base + i + s);
-          const float4* src =
-              reinterpret_cast<const float4*>(p.ws_o + (slot * kHeads + h) * kDim) + lane * 4;
+        for (int q = 0; q < 4; ++q) o[u][q] = __ldg(src + q);
+      } else {
+        m2[u] = -INFINITY;
+        l2[u] = 0.f;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) o[u][q] = __ldg(src + q);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          acc[4 * q + 0] = fmaf(wv[u], o[u][q].x, acc[4 * q + 0]);
-          acc[4 * q + 1] = fmaf(wv[u], o[u][q].y, acc[4 * q + 1]);
-          acc[4 * q + 2] = fmaf(wv[u], o[u][q].z, acc[4 * q + 2]);
-          acc[4 * q + 3] = fmaf(wv[u], o[u][q].w, acc[4 * q + 3]);
-        }
+        for (int q = 0; q < 4; ++q) o[u][q] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
-  }
+    const float Mn = fmaxf(M, fmaxf(m2[0], m2[1]));
+    const float Mu = (Mn == -INFINITY) ? 0.f : Mn;
+    const float sc = (M == -INFINITY) ? 0.f : ex2_approx(M - Mu);
+    const float w0 = (m2[0] == -INFINITY) ? 0.f : ex2_approx(m2[0] - Mu);
+    const float w1 = (m2[1] == -INFINITY) ? 0.f : ex2_approx(m2[1] - Mu);
+    L = L * sc + w0 * l2[0] + w1 * l2[1];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    for (int q = 0; q < 4; ++q) {
+      acc[4 * q + 0] = fmaf(w1, o[1][q].x, fmaf(w0, o[0][q].x, acc[4 * q + 0] * sc));
+      acc[4 * q + 1] = fmaf(w1, o[1][q].y, fmaf(w0, o[0][q].y, acc[4 * q + 1] * sc));
+      acc[4 * q + 2] = fmaf(w1, o[1][q].z, fmaf(w0, o[0][q].z, acc[4 * q + 2] * sc));
+      acc[4 * q + 3] = fmaf(w1, o[1][q].w, fmaf(w0, o[0][q].w, acc[4 * q + 3] * sc));
+    }
+    M = Mn;
+  }
   const float inv = 1.f / L;
   uint4* op = reinterpret_cast<uint4*>(out + obase);
 #pragma unroll
