@@ -164,12 +164,18 @@ def decode_workspace_size(S: int) -> int:
     return int(lib().hca_decode_workspace_size(S))
 
 
+def decode_workspace(S: int, device) -> torch.Tensor:
+    """A zero-filled decode workspace for up to S sequences (reusable across calls)."""
+    return torch.zeros((decode_workspace_size(S),), dtype=torch.uint8, device=device)
+
+
 def decode(q: torch.Tensor, ck: torch.Tensor, cv: torch.Tensor, wk: torch.Tensor,
            wv: torch.Tensor, ctx_len: torch.Tensor, g: torch.Tensor,
            scale: Optional[float] = None, workspace: Optional[torch.Tensor] = None,
            out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """One decode step: q, g [S, 64, 512]; ck, cv [S, max_nc, 512]; wk, wv
-    [S, 128, 512] ring windows; ctx_len [S] int32 on the device."""
+    [S, 128, 512] ring windows; ctx_len [S] int32 on the device.  A workspace
+    passed in comes from ``decode_workspace`` (zero-filled before first use)."""
     S, H, D = q.shape
     _check(q, "q", (S, H, HEAD_DIM))
     _check(g, "g", (S, H, HEAD_DIM))
@@ -181,9 +187,8 @@ def decode(q: torch.Tensor, ck: torch.Tensor, cv: torch.Tensor, wk: torch.Tensor
     _check(ctx_len, "ctx_len", (S,), dtype=torch.int32)
     if scale is None:
         scale = 1.0 / math.sqrt(HEAD_DIM)
-    need = decode_workspace_size(S)
     if workspace is None:
-        workspace = torch.empty((need,), dtype=torch.uint8, device=q.device)
+        workspace = decode_workspace(S, q.device)
     if out is None:
         out = torch.empty_like(q)
     _check(out, "out", (S, H, HEAD_DIM))

@@ -1,5 +1,5 @@
-// HCA decode: one new query token per sequence, split-KV over all SMs, then a
-// log-sum-exp combine.
+// HCA decode: one new query token per sequence, split-KV over all SMs, then,
+// in the same kernel behind a grid barrier, a log-sum-exp combine.
 //
 // What is computed ('BaiduがERNIE 5.5 Flash Baseを公開' §2.1; xenospectrum
 // analysis, section 活性140億パラメータと長文処理を支える仕組み): for sequence
@@ -14,6 +14,9 @@
 // A CTA writes one partial (unnormalised O, running max m, running sum l) per
 // sequence it touches, into slot c + i of the workspace (slots never collide:
 // a CTA's sequences are consecutive and later CTAs start at later sequences).
+// The launch is cooperative; after every CTA has written its partials (an
+// atomic counter, bounded spin) every CTA merges a share of the (sequence,
+// head) rows, its partial rows staged in shared memory by bulk copies.
 //
 // Tensor-core mapping (swap-AB).  With 64 heads a plain S = Q K^T would use
 // M = 64; instead keys go on the 128-lane M axis:
@@ -43,12 +46,14 @@ constexpr int kSmemRing = 65536;    // 4 x 32 KB
 constexpr int kSmemPT = kSmemRing + kStages * kStage;  // P^T [128 keys x 64 heads] bf16, 16 KB
 constexpr int kSmemRed = kSmemPT + 16384;             // reductions, 4 KB
 constexpr int kSmemBar = kSmemRed + 4096;
-constexpr int kSmemBytes = kSmemBar + 256;
+constexpr int kInlineSeqs = 1024;   // up to this many sequences each CTA plans for itself
+constexpr int kSmemTiles = kSmemBar + 256;                  // [kInlineSeqs + 1] int64 prefix
+constexpr int kSmemCtx = kSmemTiles + 8 * (kInlineSeqs + 1) + 8;  // [kInlineSeqs] int32
+constexpr int kSmemBytes = kSmemCtx + 4 * kInlineSeqs;
 constexpr int kSmemAlloc = kSmemBytes + 1024;
 constexpr int kThreads = 224;
 constexpr float kTau = 8.0f;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-constexpr int kMaxSeqs = 8192;      // prefix sums kept in shared memory? no: global scan, see below
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
 
 // reduction area layout (floats)
@@ -63,7 +68,7 @@ constexpr int R_FLAG = 768;         // ints: [0] ok, [1] any-rescale
 enum {
   B_QFULL = 0, B_QEMPTY = 1, B_FULL = 2, B_EMPTY = B_FULL + kStages, B_SFULL = B_EMPTY + kStages,
   B_SFREE = B_SFULL + 2, B_PFULL = B_SFREE + 2, B_PFREE = B_PFULL + 1, B_OFULL = B_PFREE + 1,
-  B_OFREE = B_OFULL + 1, B_DRAIN = B_OFREE + 1, B_COUNT = B_DRAIN + 1
+  B_OFREE = B_OFULL + 1, B_DRAIN = B_OFREE + 1, B_COMB = B_DRAIN + 1, B_COUNT = B_COMB + 1
 };
 constexpr int kTmemSlot = 8 * B_COUNT;
 constexpr int kAbortSlot = kTmemSlot + 4;
@@ -71,10 +76,12 @@ static_assert(kAbortSlot + 4 <= 256, "barrier region overflow");
 
 constexpr uint32_t kTmemO = 0, kTmemS0 = 256, kTmemS1 = 320, kTmemCols = 512;
 
-// Workspace layout (bytes): [slots][64][512] fp32 partial O, then [slots][2][64] fp32 (m, l)
+// Workspace layout (bytes): [slots][64 heads][128][4] bf16 partial O, normalised by its
+// l and stored with value column 128c + r at [r][c] (one 8-byte store per head
+// and TMEM lane); then [slots][2][64] fp32 (m, l)
 // in log2 units.  slots = grid + S.
 __host__ __device__ inline size_t ws_o_bytes(int slots) {
-  return static_cast<size_t>(slots) * kHeads * kDim * 4;
+  return static_cast<size_t>(slots) * kHeads * kDim * 2;
 }
 __host__ __device__ inline size_t ws_bytes(int slots) {
   return ws_o_bytes(slots) + static_cast<size_t>(slots) * 2 * kHeads * 4;
@@ -85,12 +92,23 @@ struct Params {
   int S;
   int max_nc;
   float scale_log2;
-  float* ws_o;         // [slots][64][512]
+  uint16_t* ws_o;      // [slots][64][128][4] bf16
   float* ws_ml;        // [slots][2][64]
-  long long* seq_tile; // [S + 1] exclusive prefix of tile counts (computed by plan kernel)
+  long long* seq_tile; // [S + 1] exclusive prefix of tile counts (plan kernel, S > kInlineSeqs)
+  unsigned long long* gsync;  // grid barrier arrivals (zero before first use, see below)
+  const uint16_t* g;   // [S, 64, 512] bf16 gate
+  uint16_t* out;       // [S, 64, 512] bf16
 };
 
 __device__ __forceinline__ int nc_of_len(int L) { return L >= 128 ? (L - 128) / 128 : 0; }
+
+// floor(a / b) for a >= 0, b > 0, in 32-bit arithmetic whenever both fit
+// (the 64-bit division is a long instruction sequence on the GPU).
+__device__ __forceinline__ long long div_nn(long long a, long long b) {
+  if (((static_cast<unsigned long long>(a) | static_cast<unsigned long long>(b)) >> 32) == 0)
+    return static_cast<long long>(static_cast<uint32_t>(a) / static_cast<uint32_t>(b));
+  return a / b;
+}
 
 // ---------------------------------------------------------------------------
 // Plan: tile counts per sequence and their exclusive prefix (one CTA).
@@ -145,10 +163,10 @@ struct SeqInfo {
   int L, nc, nct;   // context length, visible entries, compressed tiles
 };
 
-__device__ __forceinline__ SeqInfo seq_info(const Params& p, int s) {
+__device__ __forceinline__ SeqInfo seq_info(const int* lens, int max_nc, int s) {
   SeqInfo r;
-  r.L = max(1, p.ctx_len[s]);
-  r.nc = min(max(nc_of_len(r.L), 0), p.max_nc);
+  r.L = max(1, lens[s]);
+  r.nc = min(max(nc_of_len(r.L), 0), max_nc);
   r.nct = (r.nc + kKeyTile - 1) / kKeyTile;
   return r;
 }
@@ -161,6 +179,58 @@ __device__ __forceinline__ int find_seq(const long long* seq_tile, int S, long l
     if (seq_tile[mid] <= x) lo = mid; else hi = mid - 1;
   }
   return lo;
+}
+
+// Inline plan (S <= kInlineSeqs): every CTA reads the context lengths into
+// shared memory and computes the tile prefix itself, which saves the plan
+// kernel's launch.  Thread t takes a run of ceil(S / kThreads) sequences; the
+// runs' sums are scanned across the block.  Only CTA 0 reports bad lengths.
+__device__ __forceinline__ void inline_plan(const Params& p, long long* sT, int* sL) {
+  __shared__ long long wsum[kThreads / 32];
+  constexpr int kPer = (kInlineSeqs + kThreads - 1) / kThreads;
+  const int per = (p.S + kThreads - 1) / kThreads;
+  const int i0 = threadIdx.x * per;
+  int n[kPer];
+  long long run = 0;
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    n[u] = 0;
+    const int i = i0 + u;
+    if (u < per && i < p.S) {
+      const int L = p.ctx_len[i];
+      int nc = nc_of_len(L);
+      if ((L < 1 || nc > p.max_nc) && blockIdx.x == 0) record_error(DEVERR_BAD_INPUT, 101);
+      nc = min(max(nc, 0), p.max_nc);
+      n[u] = (nc + kKeyTile - 1) / kKeyTile + 1;
+      sL[i] = L;
+      run += n[u];
+    }
+  }
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  long long x = run;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) wsum[w] = x;
+  __syncthreads();
+  long long before = x - run;
+  for (int v = 0; v < w; ++v) before += wsum[v];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int i = i0 + u;
+    if (u < per && i < p.S) {
+      sT[i] = before;
+      before += n[u];
+    }
+  }
+  if (threadIdx.x == kThreads - 1) {
+    long long tot = 0;
+    for (int v = 0; v < kThreads / 32; ++v) tot += wsum[v];
+    sT[p.S] = tot;
+  }
+  __syncthreads();
 }
 
 // 4-D views (64, rows, 8 slabs, S) of [S][rows][512] tensors: a box
@@ -201,11 +271,254 @@ __device__ __forceinline__ void warp_transpose_reduce64(float* a) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Combine phase.  CTA c merges rows [cR/G, (c+1)R/G) of the R = 64 S
+// (sequence, head) rows, kCombRows at a time.  The partial rows a group needs
+// are, for each of its (at most two) sequences, the same head range of every
+// split that touched the sequence: contiguous runs of 2 KB per head in the
+// workspace.  They are brought into shared memory by bulk copies, together
+// with the splits' (m, l) vectors, up to kCombItems runs and the 192 KB of the
+// Q and ring buffers per batch, so a whole batch of reads is in flight at
+// once.  Everything that does not read a partial -- the group's split ranges,
+// the gate loads and sigmoid(g) -- is done before the grid barrier, while
+// the slowest CTAs are still streaming.  Warp w merges rows
+// w, w+7, w+14, w+21 of the group, the four rows interleaved: per batch the
+// largest m of its splits first, one rescale of the running sum, then one
+// weight per split; lane l covers value columns 128q + 4l .. 128q + 4l + 3
+// (q = 0..3), which keeps the shared memory reads conflict-free and the gate
+// loads and output stores 8 bytes per lane.  Empty splits (a CTA that got no
+// tile) are skipped; a split whose keys were all masked has m = -inf and
+// weight 0.
+// ---------------------------------------------------------------------------
+constexpr int kCombRows = 28;              // 7 warps x 4 rows
+constexpr int kCombItems = 32;             // runs per batch (bounded by the (m, l) area)
+constexpr int kCombData = kSmemPT;         // [Q | ring]: 192 KB of partial rows
+constexpr int kCombMl = kSmemPT;           // P^T area: 32 x 512 B of (m, l)
+static_assert(kCombItems * 512 <= 16384, "(m, l) staging area");
+
+struct CombSeq {
+  int s;       // sequence
+  int h0, nh;  // head range [h0, h0 + nh) of the group inside the sequence
+  int c0, n;   // split CTAs c0 .. c0 + n - 1
+};
+
+template <typename GridArrive, typename GridWait>
+__device__ __forceinline__ void combine_cta(const Params& p, const long long* tiles, int grid,
+                                            uint8_t* smem, uint32_t sbase, uint32_t bar_comb,
+                                            volatile int* abort_flag, int warp, int lane,
+                                            GridArrive&& grid_arrive, GridWait&& grid_wait) {
+  const long long N = tiles[p.S];
+  // CTA that owns global tile x: ceil((x + 1) * grid / N) - 1
+  auto owner = [&](long long x) -> int {
+    return static_cast<int>(div_nn((x + 1) * grid + N - 1, N)) - 1;
+  };
+  // With at least one tile per CTA every split is non-empty: the 64-bit
+  // divisions of the general test are kept off the common path.
+  const bool dense = N >= grid;
+  auto nonempty = [&](int c) { return dense || div_nn(N * c, grid) < div_nn(N * (c + 1), grid); };
+  auto seq = [&](int s, int h0, int nh) -> CombSeq {
+    CombSeq q;
+    q.s = s;
+    q.h0 = h0;
+    q.nh = nh;
+    q.c0 = owner(tiles[s]);
+    q.n = owner(tiles[s + 1] - 1) - q.c0 + 1;
+    return q;
+  };
+  const long long R = static_cast<long long>(p.S) * kHeads;
+  const long long r0 = div_nn(R * blockIdx.x, grid), r1 = div_nn(R * (blockIdx.x + 1), grid);
+  grid_arrive();  // every CTA, exactly once
+  bool waited = false;
+  uint32_t nbatch = 0;
+#pragma unroll 1
+  for (long long g0 = r0; g0 < r1; g0 += kCombRows) {
+    const int ng = static_cast<int>(min(r1 - g0, static_cast<long long>(kCombRows)));
+    const int sA = static_cast<int>(g0 / kHeads);
+    const int hA = static_cast<int>(g0 - static_cast<long long>(sA) * kHeads);
+    const int nA = min(ng, kHeads - hA);
+    const CombSeq A = seq(sA, hA, nA);
+    const CombSeq B = (ng > nA) ? seq(sA + 1, 0, ng - nA) : CombSeq{sA + 1, 0, 0, 0, 0};
+    const int nItems = A.n + B.n;
+    const uint32_t szA = static_cast<uint32_t>(A.nh) * kDim * 2;
+    const uint32_t szB = static_cast<uint32_t>(B.nh) * kDim * 2;
+
+    // this warp's rows: merge state and sigmoid(g)
+    float M[4], L[4], acc[4][16], sg[4][16];
+    {
+      // all gate loads first (rows past the group re-read its last row)
+      uint2 gv[4][4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int i = min(warp + 7 * k, ng - 1);
+        const uint2* gp = reinterpret_cast<const uint2*>(
+            p.g + static_cast<size_t>(g0 + i) * kDim + 4 * lane);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) gv[k][q4] = __ldg(gp + 32 * q4);
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        M[k] = -INFINITY;
+        L[k] = 0.f;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          acc[k][4 * q4 + 0] = acc[k][4 * q4 + 1] = acc[k][4 * q4 + 2] = acc[k][4 * q4 + 3] = 0.f;
+          sg[k][4 * q4 + 0] = sigmoid_fast(bf16lo_to_f32(gv[k][q4].x));
+          sg[k][4 * q4 + 1] = sigmoid_fast(bf16hi_to_f32(gv[k][q4].x));
+          sg[k][4 * q4 + 2] = sigmoid_fast(bf16lo_to_f32(gv[k][q4].y));
+          sg[k][4 * q4 + 3] = sigmoid_fast(bf16hi_to_f32(gv[k][q4].y));
+        }
+      }
+    }
+
+#pragma unroll 1
+    for (int fs = 0; fs < nItems;) {
+      // batch [fs, fe): at most kCombItems runs and kCombData bytes
+      int fe = fs;
+      uint32_t bytes = 0;
+      while (fe < nItems && fe - fs < kCombItems) {
+        const uint32_t sz = fe < A.n ? szA : szB;
+        if (bytes + sz > static_cast<uint32_t>(kCombData)) break;
+        bytes += sz;
+        ++fe;
+      }
+      if (!waited) {
+        grid_wait();  // every CTA's partials are written
+        waited = true;
+      }
+      if (threadIdx.x == 0) {
+        fence_proxy_async_smem();  // earlier generic reads of these buffers come first
+        uint32_t tx = 0;
+        for (int f = fs; f < fe; ++f) {
+          const bool inA = f < A.n;
+          if (nonempty(inA ? A.c0 + f : B.c0 + f - A.n)) tx += (inA ? szA : szB) + 512;
+        }
+        mbar_expect_tx(bar_comb, tx);
+        uint32_t off = 0;
+        for (int f = fs; f < fe; ++f) {
+          const bool inA = f < A.n;
+          const CombSeq& q = inA ? A : B;
+          const int c = inA ? A.c0 + f : B.c0 + f - A.n;
+          const uint32_t sz = inA ? szA : szB;
+          if (nonempty(c)) {
+            const size_t slot = static_cast<size_t>(c + q.s);
+            const uint16_t* src = p.ws_o + (slot * kHeads + q.h0) * kDim;
+            asm volatile(
+                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes"
+                " [%0], [%1], %2, [%3];" ::"r"(sbase + kSmemQ + off),
+                "l"(src), "r"(sz), "r"(bar_comb)
+                : "memory");
+            asm volatile(
+                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes"
+                " [%0], [%1], %2, [%3];" ::"r"(sbase + kCombMl + 512u * (f - fs)),
+                "l"(p.ws_ml + slot * 128), "r"(512u), "r"(bar_comb)
+                : "memory");
+          }
+          off += sz;
+        }
+      }
+      if (!mbar_wait_warp(bar_comb, nbatch & 1, abort_flag, kWaitLimitNs, 71)) return;
+      ++nbatch;
+      const int nAb = max(0, min(fe, A.n) - fs);  // runs of sequence A in this batch
+      // Per row: the batch's largest m first (lane u reads split fs + u, then a
+      // warp max), one rescale of the running sum, then one weight per split.
+      float Mb[4];
+      {
+        const int f = fs + lane;
+        const bool inA = f < A.n;
+        const bool have = f < fe && nonempty(inA ? A.c0 + f : B.c0 + f - A.n);
+        const float* ml = reinterpret_cast<const float*>(smem + kCombMl + 512 * lane);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int i = warp + 7 * k;
+          const bool rowA = i < A.nh;
+          const int h = (rowA ? A.h0 + i : i - A.nh) & 63;
+          float m = (have && rowA == inA) ? ml[h] : -INFINITY;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+          Mb[k] = fmaxf(M[k], m);
+        }
+      }
+      float Mu[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        Mu[k] = (Mb[k] == -INFINITY) ? 0.f : Mb[k];
+        const float sc = (M[k] == -INFINITY) ? 0.f : ex2_approx(M[k] - Mu[k]);
+        L[k] *= sc;
+#pragma unroll
+        for (int t = 0; t < 16; ++t) acc[k][t] *= sc;
+        M[k] = Mb[k];
+      }
+#pragma unroll 1
+      for (int f = fs; f < fe; ++f) {
+        const bool inA = f < A.n;
+        if (!nonempty(inA ? A.c0 + f : B.c0 + f - A.n)) continue;
+        const int qh0 = inA ? A.h0 : B.h0;
+        const uint32_t base = inA ? static_cast<uint32_t>(f - fs) * szA
+                                  : static_cast<uint32_t>(nAb) * szA +
+                                        static_cast<uint32_t>(f - max(fs, A.n)) * szB;
+        const float* ml = reinterpret_cast<const float*>(smem + kCombMl + 512 * (f - fs));
+        // Branch-free over the four rows (a row of the other sequence, or past
+        // the group, reads run row 0 with weight 0) so that all their shared
+        // memory reads issue together.
+        float w[4];
+        uint4 u[4][2];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int i = warp + 7 * k;
+          const bool mine = i < ng && (i < A.nh) == inA;
+          const int r = mine ? (inA ? i : i - A.nh) : 0;  // row inside this run
+          const float mi = ml[qh0 + r], li = ml[64 + qh0 + r];
+          // lane l: rows 4l + t (t = 0..3) of the [128][4] layout, i.e. value
+          // columns 128c + 4l + t, in words (t, c = 0|1) and (t, c = 2|3)
+          const uint4* row = reinterpret_cast<const uint4*>(
+              smem + kSmemQ + base + static_cast<uint32_t>(r) * kDim * 2 + 32u * lane);
+          u[k][0] = row[0];
+          u[k][1] = row[1];
+          // the partial row is normalised: its weight carries its sum l
+          w[k] = (mine && mi != -INFINITY) ? li * ex2_approx(mi - Mu[k]) : 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          L[k] += w[k];
+          const uint32_t wd[8] = {u[k][0].x, u[k][0].y, u[k][0].z, u[k][0].w,
+                                  u[k][1].x, u[k][1].y, u[k][1].z, u[k][1].w};
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            acc[k][t] = fmaf(w[k], bf16lo_to_f32(wd[2 * t]), acc[k][t]);
+            acc[k][4 + t] = fmaf(w[k], bf16hi_to_f32(wd[2 * t]), acc[k][4 + t]);
+            acc[k][8 + t] = fmaf(w[k], bf16lo_to_f32(wd[2 * t + 1]), acc[k][8 + t]);
+            acc[k][12 + t] = fmaf(w[k], bf16hi_to_f32(wd[2 * t + 1]), acc[k][12 + t]);
+          }
+        }
+      }
+      __syncthreads();  // the next batch overwrites the buffers
+      fs = fe;
+    }
+
+    // normalise, gate, store
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = warp + 7 * k;
+      if (i >= ng) continue;
+      const float inv = 1.f / L[k];
+      uint2* op = reinterpret_cast<uint2*>(p.out + static_cast<size_t>(g0 + i) * kDim + 4 * lane);
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const float* a = &acc[k][4 * q4];
+        const float* e = &sg[k][4 * q4];
+        op[32 * q4] = make_uint2(pack_bf16x2(a[0] * inv * e[0], a[1] * inv * e[1]),
+                                 pack_bf16x2(a[2] * inv * e[2], a[3] * inv * e[3]));
+      }
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ Maps maps, const Params p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned, derived from smem_raw itself so that the compiler
+  // keeps accesses through it in the shared state space
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sQ = sbase + kSmemQ, sRing = sbase + kSmemRing, sPT = sbase + kSmemPT;
   const uint32_t sBar = sbase + kSmemBar;
@@ -217,15 +530,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // The plan kernel may still be running (programmatic dependent launch):
-  // wait for its results, then let the combine kernel launch early.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const long long N = p.seq_tile[p.S];
-  const long long A0 = N * blockIdx.x / gridDim.x;
-  const long long A1 = N * (blockIdx.x + 1) / gridDim.x;
-  if (A0 >= A1) return;  // uniform across the CTA: nothing allocated yet
-
+  // Tile prefix and context lengths: planned here for up to kInlineSeqs
+  // sequences, else by the plan kernel, which may still be running
+  // (programmatic dependent launch): wait for it.
+  const bool inl = p.S <= kInlineSeqs;
+  long long* sT = reinterpret_cast<long long*>(smem + kSmemTiles);
+  int* sL = reinterpret_cast<int*>(smem + kSmemCtx);
+  if (inl) inline_plan(p, sT, sL);
+  else asm volatile("griddepcontrol.wait;" ::: "memory");
+  const long long* tiles = inl ? sT : p.seq_tile;
+  const int* lens = inl ? sL : p.ctx_len;
+  const long long N = tiles[p.S];
+  const long long A0 = div_nn(N * blockIdx.x, gridDim.x);
+  const long long A1 = div_nn(N * (blockIdx.x + 1), gridDim.x);
   if (threadIdx.x == 0) {
     mbar_init(bar(B_QFULL), 1);
     mbar_init(bar(B_QEMPTY), 1);
@@ -242,9 +559,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(B_OFULL), 1);
     mbar_init(bar(B_OFREE), 1);
     mbar_init(bar(B_DRAIN), 1);
+    mbar_init(bar(B_COMB), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
+  __syncthreads();
+  if (A0 < A1) {  // uniform across the CTA; a CTA without tiles only helps combine
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&maps.q);
     tma_prefetch_desc(&maps.ck);
@@ -262,7 +582,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   // Segments: maximal runs of this CTA's tiles inside one sequence.
-  const int s_first = find_seq(p.seq_tile, p.S, A0);
+  const int s_first = find_seq(tiles, p.S, A0);
 
   if (warp <= 1) {
     // ------------------------------------------------------------ producers
@@ -285,10 +605,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       long long x = A0;
       for (int s = s_first; x < A1 && ok; ++s) {
-        const SeqInfo si = seq_info(p, s);
-        const long long seg_end = min(A1, p.seq_tile[s + 1]);
-        const int j0 = static_cast<int>(x - p.seq_tile[s]);
-        const int j1 = static_cast<int>(seg_end - p.seq_tile[s]);
+        const SeqInfo si = seq_info(lens, p.max_nc, s);
+        const long long seg_end = min(A1, tiles[s + 1]);
+        const int j0 = static_cast<int>(x - tiles[s]);
+        const int j1 = static_cast<int>(seg_end - tiles[s]);
         if (me == 0) {
           ok = mbar_wait(bar(B_QEMPTY), (quse & 1) ^ 1, abort_flag, kWaitLimitNs, 41);
           if (!ok) break;
@@ -312,6 +632,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!load_v(j)) break;
         }
         x = seg_end;
+      }
+      // The last copies are out: bring the gate rows this CTA combines into
+      // L2 while its final tiles are processed.
+      if (me == 0) {
+        const long long R = static_cast<long long>(p.S) * kHeads;
+        const long long r0 = div_nn(R * blockIdx.x, gridDim.x);
+        const long long r1 = div_nn(R * (blockIdx.x + 1), gridDim.x);
+        if (r1 > r0)
+          asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.g + r0 * kDim),
+                       "r"(static_cast<uint32_t>(r1 - r0) * kDim * 2)
+                       : "memory");
       }
     }
   } else if (warp == 2) {
@@ -374,7 +705,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       long long x = A0;
       for (int s = s_first; x < A1 && ok; ++s) {
-        const long long seg_end = min(A1, p.seq_tile[s + 1]);
+        const long long seg_end = min(A1, tiles[s + 1]);
         const int ntl = static_cast<int>(seg_end - x);
         ok = mbar_wait(bar(B_QFULL), quse & 1, abort_flag, kWaitLimitNs, 56);
         if (!ok) break;
@@ -416,10 +747,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     long long x = A0;
     for (int s = s_first; x < A1 && ok; ++s) {
-      const SeqInfo si = seq_info(p, s);
-      const long long seg_end = min(A1, p.seq_tile[s + 1]);
-      const int j0 = static_cast<int>(x - p.seq_tile[s]);
-      const int j1 = static_cast<int>(seg_end - p.seq_tile[s]);
+      const SeqInfo si = seq_info(lens, p.max_nc, s);
+      const long long seg_end = min(A1, tiles[s + 1]);
+      const int j0 = static_cast<int>(x - tiles[s]);
+      const int j1 = static_cast<int>(seg_end - tiles[s]);
       if (tid < 64) {
         red[R_MRUN + tid] = -INFINITY;
         red[R_LRUN + tid] = 0.f;
@@ -525,20 +856,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // ---------------------------------------------------------- partial out
+      // O^T / l in bf16: this thread holds value columns 128c + key (c = 0..3)
+      // and writes them as one 8-byte word per head.
       if (!group_wait(bar(B_OFULL), nseg & 1, 62)) { ok = false; break; }
       tc_fence_after();
+      if (tid < 64) {
+        const float l = red[R_LRUN + tid];
+        red[R_ALPHA + tid] = l > 0.f ? 1.f / l : 0.f;
+      }
+      named_bar_sync(1, 128);
       const int slot = blockIdx.x + s;
-      float* wo = p.ws_o + static_cast<size_t>(slot) * kHeads * kDim;
+      uint2* wo = reinterpret_cast<uint2*>(p.ws_o + static_cast<size_t>(slot) * kHeads * kDim) + key;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int hh = 0; hh < 64; hh += 16) {
+        uint32_t o[64];
 #pragma unroll
-        for (int hh = 0; hh < 64; hh += 32) {
-          uint32_t o[32];
-          tmem_ld32(tl + kTmemO + 64 * c + hh, o);
-          tmem_wait_ld_dep32(o);
+        for (int c = 0; c < 4; ++c) tmem_ld16(tl + kTmemO + 64 * c + hh, o + 16 * c);
+        tmem_wait_ld_dep32(o);
+        reg_dep32(o + 32);
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            wo[static_cast<size_t>(hh + i) * kDim + 128 * c + key] = __uint_as_float(o[i]);
+        for (int i = 0; i < 16; ++i) {
+          const float inv = red[R_ALPHA + hh + i];
+          wo[(hh + i) * kKeyTile] =
+              make_uint2(pack_bf16x2(__uint_as_float(o[i]) * inv, __uint_as_float(o[16 + i]) * inv),
+                         pack_bf16x2(__uint_as_float(o[32 + i]) * inv,
+                                     __uint_as_float(o[48 + i]) * inv));
         }
       }
       tc_fence_before();
@@ -559,100 +901,58 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
-}
+  }  // A0 < A1
 
-// ---------------------------------------------------------------------------
-// Combine: CTA (sequence s, 8 heads), one warp per head, 16 value columns per
-// lane.  The partials are merged online (running max, rescaled accumulator),
-// two per round, so the loads of a round's (m, l) and its partial rows go out
-// together and the kernel needs few enough registers to run in one wave.
-// Empty splits are recognised arithmetically; a split whose keys were all
-// masked has m = -inf, weight 0 and a zero row.
-// ---------------------------------------------------------------------------
-constexpr int kCombineHeads = 8;
-
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
-__global__ void __launch_bounds__(32 * kCombineHeads)
-    combine_kernel(const Params p, int grid, const uint16_t* __restrict__ g,
-                   uint16_t* __restrict__ out) {
-  const int s = blockIdx.x;
-  const int h = blockIdx.y * kCombineHeads + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  // the gate row does not depend on the split pass: load it before waiting
-  const size_t obase = (static_cast<size_t>(s) * kHeads + h) * kDim + 16 * lane;
-  const uint4* gp = reinterpret_cast<const uint4*>(g + obase);
-  const uint4 gv0 = __ldg(gp), gv1 = __ldg(gp + 1);
-  pdl_wait();  // the split pass (a prerequisite grid) has finished and its writes are visible
-  const long long N = p.seq_tile[p.S];
-  const long long P0 = p.seq_tile[s], P1 = p.seq_tile[s + 1];
-  // CTA that owns global tile x: ceil((x + 1) * grid / N) - 1
-  auto owner = [&](long long x) -> int {
-    return static_cast<int>(((x + 1) * grid + N - 1) / N) - 1;
+  // ---------------------------------------------------------------- combine
+  // Grid barrier (the launch is cooperative: every CTA is resident), then the
+  // CTAs merge the partials of their share of the (sequence, head) rows.
+  // The partials are read back by bulk copies (the async proxy): every writer
+  // orders its generic stores before them.
+  // The arrival counter is never reset: every launch adds exactly gridDim.x
+  // (each CTA arrives once, on every path), so a launch's arrivals fill the
+  // window [k G, (k + 1) G) that the counter's value at its first arrival
+  // falls in, and the barrier is complete when the counter reaches (k + 1) G.
+  // It starts at zero (the workspace is zero-filled before first use) and is
+  // 64-bit, so it does not wrap.
+  __shared__ unsigned long long bar_target;
+  __shared__ int bar_done;
+  auto grid_arrive = [&]() {
+    fence_proxy_async_all();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      // acq_rel: releases this CTA's partials (ordered before it by the CTA
+      // barrier above); the last arrival also acquires everybody else's and
+      // so needs no polling
+      const unsigned long long G = gridDim.x;
+      unsigned long long old;
+      asm volatile("atom.add.acq_rel.gpu.global.u64 %0, [%1], 1;"
+                   : "=l"(old)
+                   : "l"(p.gsync)
+                   : "memory");
+      bar_target = (old / G + 1) * G;
+      bar_done = (old + 1 == bar_target) ? 1 : 0;
+    }
   };
-  const int c0 = owner(P0), c1 = owner(P1 - 1);
-  const int np = c1 - c0 + 1;
-  auto nonempty = [&](int c) { return N * c / grid < N * (c + 1) / grid; };
-  float acc[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-  float M = -INFINITY, L = 0.f;
-#pragma unroll 1
-  for (int i0 = 0; i0 < np; i0 += 2) {
-    float m2[2], l2[2];
-    float4 o[2][4];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int c = c0 + i0 + u;
-      if (i0 + u < np && nonempty(c)) {
-        const size_t slot = static_cast<size_t>(c + s);
-        m2[u] = __ldg(p.ws_ml + slot * 128 + h);
-        l2[u] = __ldg(p.ws_ml + slot * 128 + 64 + h);
-        const float4* src =
-            reinterpret_cast<const float4*>(p.ws_o + (slot * kHeads + h) * kDim) + lane * 4;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) o[u][q] = __ldg(src + q);
-      } else {
-        m2[u] = -INFINITY;
-        l2[u] = 0.f;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) o[u][q] = make_float4(0.f, 0.f, 0.f, 0.f);
+  auto grid_wait = [&]() {
+    if (threadIdx.x == 0 && !bar_done) {
+      const uint64_t t0 = globaltimer_ns();
+      for (uint32_t i = 1;; ++i) {
+        unsigned long long v;
+        asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p.gsync) : "memory");
+        if (v >= bar_target) break;
+        if ((i & 63u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+          record_error(DEVERR_TIMEOUT, 70);
+          break;
+        }
       }
     }
-    const float Mn = fmaxf(M, fmaxf(m2[0], m2[1]));
-    const float Mu = (Mn == -INFINITY) ? 0.f : Mn;
-    const float sc = (M == -INFINITY) ? 0.f : ex2_approx(M - Mu);
-    const float w0 = (m2[0] == -INFINITY) ? 0.f : ex2_approx(m2[0] - Mu);
-    const float w1 = (m2[1] == -INFINITY) ? 0.f : ex2_approx(m2[1] - Mu);
-    L = L * sc + w0 * l2[0] + w1 * l2[1];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      acc[4 * q + 0] = fmaf(w1, o[1][q].x, fmaf(w0, o[0][q].x, acc[4 * q + 0] * sc));
-      acc[4 * q + 1] = fmaf(w1, o[1][q].y, fmaf(w0, o[0][q].y, acc[4 * q + 1] * sc));
-      acc[4 * q + 2] = fmaf(w1, o[1][q].z, fmaf(w0, o[0][q].z, acc[4 * q + 2] * sc));
-      acc[4 * q + 3] = fmaf(w1, o[1][q].w, fmaf(w0, o[0][q].w, acc[4 * q + 3] * sc));
-    }
-    M = Mn;
-  }
-  const float inv = 1.f / L;
-  uint4* op = reinterpret_cast<uint4*>(out + obase);
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    const uint4 gv = q ? gv1 : gv0;
-    const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-    uint32_t ow[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float a0 = acc[8 * q + 2 * k] * inv * sigmoid_fast(bf16lo_to_f32(gw[k]));
-      const float a1 = acc[8 * q + 2 * k + 1] * inv * sigmoid_fast(bf16hi_to_f32(gw[k]));
-      ow[k] = pack_bf16x2(a0, a1);
-    }
-    op[q] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-  }
+    if (threadIdx.x == 0) fence_proxy_async_all();
+    __syncthreads();
+  };
+  combine_cta(p, tiles, gridDim.x, smem, sbase, bar(B_COMB), abort_flag, warp, lane,
+              grid_arrive, grid_wait);
 }
 
+// ---------------------------------------------------------------------------
 }  // namespace decode
 }  // namespace hca

@@ -103,23 +103,35 @@ int prefill_max_pairs() {
   return cached;
 }
 
-// Launch `kernel` on `stream` allowing programmatic dependent launch: it may
-// start while the previous kernel on the stream is still running, and waits
-// for it inside (griddepcontrol.wait).
-template <typename... Params, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
-                       cudaStream_t stream, Args&&... args) {
+// The decode pass: for more than kInlineSeqs sequences the plan kernel first
+// (the decode kernel then starts early and waits for it inside), else the
+// decode kernel alone, which plans for itself.  Cooperative either way: the
+// kernel holds a grid barrier.
+cudaError_t launch_decode(const hca::decode::Maps& maps, const hca::decode::Params& prm, int grid,
+                          cudaStream_t stream) {
+  namespace D = hca::decode;
+  cudaError_t err = cudaFuncSetAttribute(D::decode_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, D::kSmemAlloc);
+  if (err != cudaSuccess) return err;
+  const bool inl = prm.S <= D::kInlineSeqs;
+  if (!inl) {
+    D::plan_kernel<<<1, 1024, 0, stream>>>(prm.ctx_len, prm.S, prm.max_nc, prm.seq_tile);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(D::kThreads);
+  cfg.dynamicSmemBytes = D::kSmemAlloc;
   cfg.stream = stream;
-  cudaLaunchAttribute attr;
-  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr.val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = &attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = inl ? 1 : 2;
+  return cudaLaunchKernelEx(&cfg, D::decode_kernel, maps, prm);
 }
 
 hca_status_t launch_status() {
@@ -234,8 +246,9 @@ size_t hca_decode_workspace_size(int S) {
   const int sms = device_sms();
   if (sms <= 0) return 0;
   const int slots = sms + S;
-  // partial O and (m, l) per slot, then the tile prefix [S + 1] int64
-  return hca::decode::ws_bytes(slots) + 256 + static_cast<size_t>(S + 1) * 8;
+  // the grid barrier counter (256-byte block at offset 0), partial O and
+  // (m, l) per slot, then the tile prefix [S + 1] int64
+  return 256 + hca::decode::ws_bytes(slots) + 256 + static_cast<size_t>(S + 1) * 8;
 }
 
 hca_status_t hca_decode(const hca_bf16* q, const hca_bf16* ck, const hca_bf16* cv, int max_nc,
@@ -266,9 +279,13 @@ hca_status_t hca_decode(const hca_bf16* q, const hca_bf16* ck, const hca_bf16* c
   prm.S = S;
   prm.max_nc = max_nc;
   prm.scale_log2 = scale * 1.4426950408889634f;
-  prm.ws_o = reinterpret_cast<float*>(wsb);
-  prm.ws_ml = reinterpret_cast<float*>(wsb + D::ws_o_bytes(slots));
-  prm.seq_tile = reinterpret_cast<long long*>(wsb + ((D::ws_bytes(slots) + 255) & ~size_t(255)));
+  prm.gsync = reinterpret_cast<unsigned long long*>(wsb);
+  prm.ws_o = reinterpret_cast<uint16_t*>(wsb + 256);
+  prm.ws_ml = reinterpret_cast<float*>(wsb + 256 + D::ws_o_bytes(slots));
+  prm.seq_tile =
+      reinterpret_cast<long long*>(wsb + 256 + ((D::ws_bytes(slots) + 255) & ~size_t(255)));
+  prm.g = g;
+  prm.out = out;
 
   D::Maps maps;
   bool ok = make_map4(&maps.q, q, static_cast<uint64_t>(S) * HCA_NUM_HEADS, 1, 64, 8) &&
@@ -282,17 +299,7 @@ hca_status_t hca_decode(const hca_bf16* q, const hca_bf16* ck, const hca_bf16* c
   }
   if (!ok) return HCA_ERR_CUDA;
 
-  D::plan_kernel<<<1, 1024, 0, stream>>>(ctx_len, S, max_nc, prm.seq_tile);
-  if (cudaGetLastError() != cudaSuccess) return HCA_ERR_CUDA;
-  if (cudaFuncSetAttribute(D::decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           D::kSmemAlloc) != cudaSuccess)
-    return HCA_ERR_CUDA;
-  if (launch_pdl(D::decode_kernel, dim3(sms), dim3(D::kThreads), D::kSmemAlloc, stream, maps,
-                 prm) != cudaSuccess)
-    return HCA_ERR_CUDA;
-  if (launch_pdl(D::combine_kernel, dim3(S, HCA_NUM_HEADS / D::kCombineHeads),
-                 dim3(32 * D::kCombineHeads), 0, stream, prm, sms, g, out) != cudaSuccess)
-    return HCA_ERR_CUDA;
+  if (launch_decode(maps, prm, sms, stream) != cudaSuccess) return HCA_ERR_CUDA;
   return launch_status();
 }
 
@@ -305,14 +312,15 @@ hca_status_t hca_decode(const hca_bf16* q, const hca_bf16* ck, const hca_bf16* c
 namespace {
 
 constexpr int kNoAllocSlots = HCA_NOALLOC_MAX_CTAS + HCA_NOALLOC_MAX_SEQS;
-// per slot: partial O [64][512] fp32 + (m, l) [2][64] fp32
-constexpr size_t kNoAllocSlotBytes = static_cast<size_t>(64) * 512 * 4 + 2 * 64 * 4;
+// per slot: partial O [64][512] bf16 + (m, l) [2][64] fp32
+constexpr size_t kNoAllocSlotBytes = static_cast<size_t>(64) * 512 * 2 + 2 * 64 * 4;
 constexpr size_t kNoAllocPrefixOffset =
-    (kNoAllocSlots * kNoAllocSlotBytes + 255) & ~static_cast<size_t>(255);
+    256 + ((kNoAllocSlots * kNoAllocSlotBytes + 255) & ~static_cast<size_t>(255));
 constexpr size_t kNoAllocScratchBytes =
     kNoAllocPrefixOffset + static_cast<size_t>(HCA_NOALLOC_MAX_SEQS + 1) * 8;
 
-// Partial O / (m, l) of up to kNoAllocSlots split slots, then the tile prefix.
+// The grid barrier counter (zero at load), partial O / (m, l) of up to
+// kNoAllocSlots split slots, then the tile prefix.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxDevices = 64;
@@ -365,9 +373,12 @@ hca_status_t hca_decode_noalloc(const hca_bf16* q, const hca_bf16* ck, const hca
   prm.S = S;
   prm.max_nc = max_nc;
   prm.scale_log2 = scale * 1.4426950408889634f;
-  prm.ws_o = reinterpret_cast<float*>(wsb);
-  prm.ws_ml = reinterpret_cast<float*>(wsb + D::ws_o_bytes(slots));
+  prm.gsync = reinterpret_cast<unsigned long long*>(wsb);
+  prm.ws_o = reinterpret_cast<uint16_t*>(wsb + 256);
+  prm.ws_ml = reinterpret_cast<float*>(wsb + 256 + D::ws_o_bytes(slots));
   prm.seq_tile = reinterpret_cast<long long*>(wsb + kNoAllocPrefixOffset);
+  prm.g = g;
+  prm.out = out;
 
   D::Maps maps;
   bool ok = make_map4(&maps.q, q, static_cast<uint64_t>(S) * HCA_NUM_HEADS, 1, 64, 8) &&
@@ -381,17 +392,7 @@ hca_status_t hca_decode_noalloc(const hca_bf16* q, const hca_bf16* ck, const hca
   }
   if (!ok) return HCA_ERR_CUDA;
 
-  D::plan_kernel<<<1, 1024, 0, stream>>>(ctx_len, S, max_nc, prm.seq_tile);
-  if (cudaGetLastError() != cudaSuccess) return HCA_ERR_CUDA;
-  if (cudaFuncSetAttribute(D::decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           D::kSmemAlloc) != cudaSuccess)
-    return HCA_ERR_CUDA;
-  if (launch_pdl(D::decode_kernel, dim3(grid), dim3(D::kThreads), D::kSmemAlloc, stream, maps,
-                 prm) != cudaSuccess)
-    return HCA_ERR_CUDA;
-  if (launch_pdl(D::combine_kernel, dim3(S, HCA_NUM_HEADS / D::kCombineHeads),
-                 dim3(32 * D::kCombineHeads), 0, stream, prm, grid, g, out) != cudaSuccess)
-    return HCA_ERR_CUDA;
+  if (launch_decode(maps, prm, grid, stream) != cudaSuccess) return HCA_ERR_CUDA;
   return launch_status();
 }
 

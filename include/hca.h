@@ -105,7 +105,10 @@ hca_status_t hca_prefill_fwd(const hca_bf16* q, const hca_bf16* k, const hca_bf1
 
 /*
  * hca_decode_workspace_size — bytes of scratch hca_decode needs for S
- * sequences on the current device (partial results of the split-KV pass).
+ * sequences on the current device (partial results of the split-KV pass and
+ * a grid-barrier counter).  A workspace must be zero-filled once before its
+ * first hca_decode call (e.g. cudaMemsetAsync); every call leaves it valid for
+ * the next one, whatever S, on the same device.
  */
 size_t hca_decode_workspace_size(int S);
 
@@ -122,7 +125,8 @@ size_t hca_decode_workspace_size(int S);
  * Layout:  q, g, out [S, H, 512] bf16 (H = 64);  ck, cv [S, max_nc, 512] bf16;
  *          wk, wv [S, 128, 512] bf16;  ctx_len [S] int32 on the device;
  *          ws: caller-owned device scratch of at least
- *          hca_decode_workspace_size(S) bytes, 256-byte aligned.
+ *          hca_decode_workspace_size(S) bytes, 256-byte aligned, zero-filled
+ *          before its first use; one call at a time per workspace.
  * Errors:  host-checked as for prefill (and ws_bytes too small ->
  *          HCA_ERR_INVALID_ARG).  A device-side ctx_len < 1 or one needing more
  *          than max_nc entries is clamped and reported later by

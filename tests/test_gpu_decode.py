@@ -106,3 +106,45 @@ def test_decode_bad_device_length_is_reported_not_faulted():
     code, _ = hca.device_error()
     assert code == 5  # HCA_ERR_DEVICE_INPUT
     assert hca.device_error()[0] == 0  # cleared
+
+
+def test_decode_many_sequences_planned_by_plan_kernel():
+    """More sequences than one CTA plans for itself: the tile prefix then comes
+    from the separate plan kernel."""
+    need_gpu()
+    rng = np.random.default_rng(11)
+    lens = [int(x) for x in rng.integers(1, 700, size=1100)]
+    max_nc = 4
+    q, g, ck, cv, wk, wv = _direct_case(lens, max_nc, seed=12)
+    out = _run(q, g, ck, cv, wk, wv, lens)
+    ref = O.decode_forward(to64(q), to64(ck), to64(cv), to64(wk), to64(wv), lens, to64(g))
+    assert_close_out(to64(out), ref, "S=1100")
+
+
+def test_decode_workspace_reused_across_calls_and_sizes():
+    """One zero-filled workspace serves many calls of different S: the grid
+    barrier's counter is never reset, so a wrong window would show up as a
+    race (different results) on some call."""
+    need_gpu()
+    ws = hca.decode_workspace(64, torch.device("cuda"))
+    cases = []
+    for lens, seed in (([3000, 129, 700, 5000, 1], 21), ([20000] * 2 + [300] * 62, 22)):
+        max_nc = max(1, max(max(0, (L - 128) // 128) for L in lens))
+        args = [t.cuda() for t in _direct_case(lens, max_nc, seed)]
+        ctx = torch.tensor(lens, dtype=torch.int32, device="cuda")
+        cases.append((args, ctx, lens))
+    first = []
+    for rep in range(12):
+        for ci, (args, ctx, lens) in enumerate(cases):
+            q, g, ck, cv, wk, wv = args
+            out = hca.decode(q, ck, cv, wk, wv, ctx, g, workspace=ws)
+            torch.cuda.synchronize()
+            if rep == 0:
+                first.append(out.clone())
+                ref = O.decode_forward(to64(q), to64(ck), to64(cv), to64(wk), to64(wv), lens,
+                                       to64(g))
+                assert_close_out(to64(out), ref, f"case {ci}")
+            else:
+                assert torch.equal(out, first[ci]), f"case {ci} rep {rep} differs"
+    code, where = hca.device_error()
+    assert code == 0, f"device error {code} at {where}"
