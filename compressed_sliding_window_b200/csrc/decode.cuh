@@ -296,11 +296,89 @@ constexpr int kCombData = kSmemPT;         // [Q | ring]: 192 KB of partial rows
 constexpr int kCombMl = kSmemPT;           // P^T area: 32 x 512 B of (m, l)
 static_assert(kCombItems * 512 <= 16384, "(m, l) staging area");
 
+// sigmoid(g) is held as f16 pairs until the store (its relative rounding,
+// 2^-11, is below that of the bf16 output)
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ float f16lo_to_f32(uint32_t v) {
+  float r;
+  asm("{.reg .f16 a, b;\n mov.b32 {a, b}, %1;\n cvt.f32.f16 %0, a;}" : "=f"(r) : "r"(v));
+  return r;
+}
+__device__ __forceinline__ float f16hi_to_f32(uint32_t v) {
+  float r;
+  asm("{.reg .f16 a, b;\n mov.b32 {a, b}, %1;\n cvt.f32.f16 %0, b;}" : "=f"(r) : "r"(v));
+  return r;
+}
+
 struct CombSeq {
   int s;       // sequence
   int h0, nh;  // head range [h0, h0 + nh) of the group inside the sequence
   int c0, n;   // split CTAs c0 .. c0 + n - 1
 };
+
+// Merge of one batch's runs into a warp's first NK rows, NU runs per step
+// (NK x NU <= 4 row-runs in flight per step).  Runs are taken in order;
+// `run_of(f)` gives run f's byte offset in the staged buffer and whether it
+// holds data (an empty split's run was never copied), `seq_a(f)` whether run
+// f belongs to the group's first sequence.  A row of the other sequence reads
+// some in-bounds words and replaces them by zeros with weight 0.
+template <int NK, int NU, typename RunOf, typename SeqA>
+__device__ __forceinline__ void merge_runs(const uint8_t* smem, int fs, int fe,
+                                           const bool (&rowA)[4], const int (&hrow)[4],
+                                           const uint32_t (&roff)[4], const float (&Mu)[4],
+                                           float (&L)[4], float (&acc)[4][16], RunOf&& run_of,
+                                           SeqA&& seq_a) {
+#pragma unroll 1
+  for (int f = fs; f < fe; f += NU) {
+    uint4 x[NU][NK][2];
+    float w[NU][NK];
+#pragma unroll
+    for (int u = 0; u < NU; ++u) {
+      const int fu = min(f + u, fe - 1);
+      bool live;
+      const uint32_t base = run_of(fu, live);
+      live = live && f + u < fe;
+      const bool inA = seq_a(fu);
+      const float* ml = reinterpret_cast<const float*>(smem + kCombMl + 512 * (fu - fs));
+#pragma unroll
+      for (int k = 0; k < NK; ++k) {
+        const uint4* row = reinterpret_cast<const uint4*>(smem + kSmemQ + base + roff[k]);
+        x[u][k][0] = row[0];
+        x[u][k][1] = row[1];
+        const float mi = ml[hrow[k]], li = ml[64 + hrow[k]];
+        // the partial row is normalised: its weight carries its sum l
+        const bool mine = live && rowA[k] == inA;
+        w[u][k] = (mine && mi != -INFINITY) ? li * ex2_approx(mi - Mu[k]) : 0.f;
+        if (!mine) {  // not this row's data (or never copied): may hold anything
+          x[u][k][0] = make_uint4(0u, 0u, 0u, 0u);
+          x[u][k][1] = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+    }
+    // lane l: rows 4l + t (t = 0..3) of the [128][4] layout, i.e. value
+    // columns 128c + 4l + t, in words (t, c = 0|1) and (t, c = 2|3)
+#pragma unroll
+    for (int k = 0; k < NK; ++k) {
+#pragma unroll
+      for (int u = 0; u < NU; ++u) {
+        L[k] += w[u][k];
+        const uint32_t wd[8] = {x[u][k][0].x, x[u][k][0].y, x[u][k][0].z, x[u][k][0].w,
+                                x[u][k][1].x, x[u][k][1].y, x[u][k][1].z, x[u][k][1].w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          acc[k][t] = fmaf(w[u][k], bf16lo_to_f32(wd[2 * t]), acc[k][t]);
+          acc[k][4 + t] = fmaf(w[u][k], bf16hi_to_f32(wd[2 * t]), acc[k][4 + t]);
+          acc[k][8 + t] = fmaf(w[u][k], bf16lo_to_f32(wd[2 * t + 1]), acc[k][8 + t]);
+          acc[k][12 + t] = fmaf(w[u][k], bf16hi_to_f32(wd[2 * t + 1]), acc[k][12 + t]);
+        }
+      }
+    }
+  }
+}
 
 template <typename GridArrive, typename GridWait>
 __device__ __forceinline__ void combine_cta(const Params& p, const long long* tiles, int grid,
@@ -343,7 +421,8 @@ __device__ __forceinline__ void combine_cta(const Params& p, const long long* ti
     const uint32_t szB = static_cast<uint32_t>(B.nh) * kDim * 2;
 
     // this warp's rows: merge state and sigmoid(g)
-    float M[4], L[4], acc[4][16], sg[4][16];
+    float M[4], L[4], acc[4][16];
+    uint32_t sg[4][8];
     {
       // all gate loads first (rows past the group re-read its last row)
       uint2 gv[4][4];
@@ -362,10 +441,10 @@ __device__ __forceinline__ void combine_cta(const Params& p, const long long* ti
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           acc[k][4 * q4 + 0] = acc[k][4 * q4 + 1] = acc[k][4 * q4 + 2] = acc[k][4 * q4 + 3] = 0.f;
-          sg[k][4 * q4 + 0] = sigmoid_fast(bf16lo_to_f32(gv[k][q4].x));
-          sg[k][4 * q4 + 1] = sigmoid_fast(bf16hi_to_f32(gv[k][q4].x));
-          sg[k][4 * q4 + 2] = sigmoid_fast(bf16lo_to_f32(gv[k][q4].y));
-          sg[k][4 * q4 + 3] = sigmoid_fast(bf16hi_to_f32(gv[k][q4].y));
+          sg[k][2 * q4] = pack_f16x2(sigmoid_fast(bf16lo_to_f32(gv[k][q4].x)),
+                                     sigmoid_fast(bf16hi_to_f32(gv[k][q4].x)));
+          sg[k][2 * q4 + 1] = pack_f16x2(sigmoid_fast(bf16lo_to_f32(gv[k][q4].y)),
+                                         sigmoid_fast(bf16hi_to_f32(gv[k][q4].y)));
         }
       }
     }
@@ -448,49 +527,37 @@ __device__ __forceinline__ void combine_cta(const Params& p, const long long* ti
         for (int t = 0; t < 16; ++t) acc[k][t] *= sc;
         M[k] = Mb[k];
       }
-#pragma unroll 1
-      for (int f = fs; f < fe; ++f) {
-        const bool inA = f < A.n;
-        if (!nonempty(inA ? A.c0 + f : B.c0 + f - A.n)) continue;
-        const int qh0 = inA ? A.h0 : B.h0;
-        const uint32_t base = inA ? static_cast<uint32_t>(f - fs) * szA
-                                  : static_cast<uint32_t>(nAb) * szA +
-                                        static_cast<uint32_t>(f - max(fs, A.n)) * szB;
-        const float* ml = reinterpret_cast<const float*>(smem + kCombMl + 512 * (f - fs));
-        // Branch-free over the four rows (a row of the other sequence, or past
-        // the group, reads run row 0 with weight 0) so that all their shared
-        // memory reads issue together.
-        float w[4];
-        uint4 u[4][2];
+      // The warp's rows (k < nk) with a loop specialised to their count, so
+      // that no read is spent on a row past the group and a single row still
+      // has several runs in flight.
+      bool rowA[4];
+      int hrow[4];
+      uint32_t roff[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int i = warp + 7 * k;
-          const bool mine = i < ng && (i < A.nh) == inA;
-          const int r = mine ? (inA ? i : i - A.nh) : 0;  // row inside this run
-          const float mi = ml[qh0 + r], li = ml[64 + qh0 + r];
-          // lane l: rows 4l + t (t = 0..3) of the [128][4] layout, i.e. value
-          // columns 128c + 4l + t, in words (t, c = 0|1) and (t, c = 2|3)
-          const uint4* row = reinterpret_cast<const uint4*>(
-              smem + kSmemQ + base + static_cast<uint32_t>(r) * kDim * 2 + 32u * lane);
-          u[k][0] = row[0];
-          u[k][1] = row[1];
-          // the partial row is normalised: its weight carries its sum l
-          w[k] = (mine && mi != -INFINITY) ? li * ex2_approx(mi - Mu[k]) : 0.f;
-        }
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          L[k] += w[k];
-          const uint32_t wd[8] = {u[k][0].x, u[k][0].y, u[k][0].z, u[k][0].w,
-                                  u[k][1].x, u[k][1].y, u[k][1].z, u[k][1].w};
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            acc[k][t] = fmaf(w[k], bf16lo_to_f32(wd[2 * t]), acc[k][t]);
-            acc[k][4 + t] = fmaf(w[k], bf16hi_to_f32(wd[2 * t]), acc[k][4 + t]);
-            acc[k][8 + t] = fmaf(w[k], bf16lo_to_f32(wd[2 * t + 1]), acc[k][8 + t]);
-            acc[k][12 + t] = fmaf(w[k], bf16hi_to_f32(wd[2 * t + 1]), acc[k][12 + t]);
-          }
-        }
+      for (int k = 0; k < 4; ++k) {
+        const int i = min(warp + 7 * k, ng - 1);
+        rowA[k] = i < A.nh;
+        const int r = rowA[k] ? i : i - A.nh;
+        hrow[k] = (rowA[k] ? A.h0 : B.h0) + r;
+        roff[k] = static_cast<uint32_t>(r) * kDim * 2 + 32u * lane;
       }
+      auto run_of = [&](int f, bool& live) -> uint32_t {
+        const bool inA = f < A.n;
+        live = nonempty(inA ? A.c0 + f : B.c0 + f - A.n);
+        return inA ? static_cast<uint32_t>(f - fs) * szA
+                   : static_cast<uint32_t>(nAb) * szA +
+                         static_cast<uint32_t>(f - max(fs, A.n)) * szB;
+      };
+      auto seq_a = [&](int f) { return f < A.n; };
+      const int nk = ng > warp ? min(4, (ng - warp + 6) / 7) : 0;
+      if (nk == 4)
+        merge_runs<4, 1>(smem, fs, fe, rowA, hrow, roff, Mu, L, acc, run_of, seq_a);
+      else if (nk == 3)
+        merge_runs<3, 1>(smem, fs, fe, rowA, hrow, roff, Mu, L, acc, run_of, seq_a);
+      else if (nk == 2)
+        merge_runs<2, 2>(smem, fs, fe, rowA, hrow, roff, Mu, L, acc, run_of, seq_a);
+      else if (nk == 1)
+        merge_runs<1, 4>(smem, fs, fe, rowA, hrow, roff, Mu, L, acc, run_of, seq_a);
       __syncthreads();  // the next batch overwrites the buffers
       fs = fe;
     }
@@ -505,9 +572,10 @@ __device__ __forceinline__ void combine_cta(const Params& p, const long long* ti
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         const float* a = &acc[k][4 * q4];
-        const float* e = &sg[k][4 * q4];
-        op[32 * q4] = make_uint2(pack_bf16x2(a[0] * inv * e[0], a[1] * inv * e[1]),
-                                 pack_bf16x2(a[2] * inv * e[2], a[3] * inv * e[3]));
+        const uint32_t e01 = sg[k][2 * q4], e23 = sg[k][2 * q4 + 1];
+        op[32 * q4] = make_uint2(
+            pack_bf16x2(a[0] * inv * f16lo_to_f32(e01), a[1] * inv * f16hi_to_f32(e01)),
+            pack_bf16x2(a[2] * inv * f16lo_to_f32(e23), a[3] * inv * f16hi_to_f32(e23)));
       }
     }
   }
