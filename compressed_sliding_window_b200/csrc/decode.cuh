@@ -598,19 +598,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // Tile prefix and context lengths: planned here for up to kInlineSeqs
-  // sequences, else by the plan kernel, which may still be running
-  // (programmatic dependent launch): wait for it.
-  const bool inl = p.S <= kInlineSeqs;
-  long long* sT = reinterpret_cast<long long*>(smem + kSmemTiles);
-  int* sL = reinterpret_cast<int*>(smem + kSmemCtx);
-  if (inl) inline_plan(p, sT, sL);
-  else asm volatile("griddepcontrol.wait;" ::: "memory");
-  const long long* tiles = inl ? sT : p.seq_tile;
-  const int* lens = inl ? sL : p.ctx_len;
-  const long long N = tiles[p.S];
-  const long long A0 = div_nn(N * blockIdx.x, gridDim.x);
-  const long long A1 = div_nn(N * (blockIdx.x + 1), gridDim.x);
+  // Set-up that needs no plan first, so that it overlaps the plan's loads:
+  // barriers, tensor-map prefetch, TMEM.
   if (threadIdx.x == 0) {
     mbar_init(bar(B_QFULL), 1);
     mbar_init(bar(B_QEMPTY), 1);
@@ -630,10 +619,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(B_COMB), 1);
     *abort_flag = 0;
     fence_mbar_init();
-  }
-  __syncthreads();
-  if (A0 < A1) {  // uniform across the CTA; a CTA without tiles only helps combine
-  if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&maps.q);
     tma_prefetch_desc(&maps.ck);
     tma_prefetch_desc(&maps.cv);
@@ -645,9 +630,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
     tc_fence_before();
   }
-  __syncthreads();
+  // Tile prefix and context lengths: planned here for up to kInlineSeqs
+  // sequences, else by the plan kernel, which may still be running
+  // (programmatic dependent launch): wait for it.  Either way a CTA barrier
+  // follows, which also publishes the set-up above.
+  const bool inl = p.S <= kInlineSeqs;
+  long long* sT = reinterpret_cast<long long*>(smem + kSmemTiles);
+  int* sL = reinterpret_cast<int*>(smem + kSmemCtx);
+  if (inl) {
+    inline_plan(p, sT, sL);
+  } else {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    __syncthreads();
+  }
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const long long* tiles = inl ? sT : p.seq_tile;
+  const int* lens = inl ? sL : p.ctx_len;
+  const long long N = tiles[p.S];
+  const long long A0 = div_nn(N * blockIdx.x, gridDim.x);
+  const long long A1 = div_nn(N * (blockIdx.x + 1), gridDim.x);
+  if (A0 < A1) {  // uniform across the CTA; a CTA without tiles only helps combine
 
   // Segments: maximal runs of this CTA's tiles inside one sequence.
   const int s_first = find_seq(tiles, p.S, A0);
@@ -964,12 +967,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  }  // A0 < A1
   __syncthreads();
   if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
-  }  // A0 < A1
 
   // ---------------------------------------------------------------- combine
   // Grid barrier (the launch is cooperative: every CTA is resident), then the
