@@ -469,6 +469,39 @@ __device__ __forceinline__ float sigmoid_fast(float x) {
   return fmaf(0.5f, tanh_approx(0.5f * x), 0.5f);
 }
 
+__device__ __forceinline__ uint32_t pack_bf16x2_fwd(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Gated output pair, out = o * il * sigmoid(g) for two columns, written as
+// h (1 + tanh(g / 2)) with h = o * (il / 2): two MUFU ops and three packed
+// f32x2 operations (sm_100) per pair.  hil = il / 2; g is a bf16 pair.
+__device__ __forceinline__ uint32_t gate_pair_bf16(float o0, float o1, float hil, uint32_t g) {
+  const float gl = __uint_as_float(g << 16), gh = __uint_as_float(g & 0xffff0000u);
+  float xl, xh;
+  asm("{.reg .b64 gp, hp, xp;\n"
+      " mov.b64 gp, {%2, %3};\n"
+      " mov.b64 hp, {%4, %4};\n"
+      " mul.rn.f32x2 xp, gp, hp;\n"
+      " mov.b64 {%0, %1}, xp;}"
+      : "=f"(xl), "=f"(xh)
+      : "f"(gl), "f"(gh), "f"(0.5f));
+  const float tl = tanh_approx(xl), th = tanh_approx(xh);
+  float rl, rh;
+  asm("{.reg .b64 op, hp, hh, tp, rp;\n"
+      " mov.b64 op, {%2, %3};\n"
+      " mov.b64 hp, {%4, %4};\n"
+      " mul.rn.f32x2 hh, op, hp;\n"
+      " mov.b64 tp, {%5, %6};\n"
+      " fma.rn.f32x2 rp, hh, tp, hh;\n"
+      " mov.b64 {%0, %1}, rp;}"
+      : "=f"(rl), "=f"(rh)
+      : "f"(o0), "f"(o1), "f"(hil), "f"(tl), "f"(th));
+  return pack_bf16x2_fwd(rl, rh);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

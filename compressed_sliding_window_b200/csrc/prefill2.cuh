@@ -735,6 +735,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const float il = invl_s[row];
+        const float hil = 0.5f * il;
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(peerStatsFree);
         const uint32_t gbase = ubase + v_uses(x);
@@ -774,9 +775,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
                 const int oc = 8 * c4 + 2 * q;
-                ow[q] = pack_bf16x2(__uint_as_float(o[oc]) * il * sigmoid_fast(bf16lo_to_f32(gw[q])),
-                                    __uint_as_float(o[oc + 1]) * il *
-                                        sigmoid_fast(bf16hi_to_f32(gw[q])));
+                ow[q] = gate_pair_bf16(__uint_as_float(o[oc]), __uint_as_float(o[oc + 1]), hil,
+                                       gw[q]);
               }
               *ptr = make_uint4(ow[0], ow[1], ow[2], ow[3]);
             }
