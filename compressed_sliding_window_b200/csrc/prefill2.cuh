@@ -81,7 +81,7 @@ enum {
   SFREE = SFULL + 2, PFREE = SFREE + 2, STATSFREE = PFREE + 4,
   VFULL = STATSFREE + 1, VEMPTY = VFULL + kVStages, PREADY = VEMPTY + kVStages,
   PFULL = PREADY + 4, PBUFFREE = PFULL + 2, CORR = PBUFFREE + 2,
-  PVDONE = CORR + 2, OFULL = PVDONE + 2, OFREE = OFULL + 1, STATSFULL = OFREE + 2,
+  PVDONE = CORR + 2, OFULL = PVDONE + 2, OFREE = OFULL + 2, STATSFULL = OFREE + 2,
   STAGED = STATSFULL + 1, DRAIN = STAGED + 4, NBAR = DRAIN + 1
 };
 constexpr int kTmemSlot = BAR + 8 * NBAR;
@@ -155,17 +155,18 @@ __device__ __forceinline__ int sub_n(int n, int h) { return h == 0 ? min(n, 128)
 
 // P.V order of one tile, walked by both the V producer and the MMA issuer:
 // step s of 2 * nkt (nkt = 64-key chunks of both sub-tiles, nk0 of them in
-// sub-tile 0) -> value half dh, sub-tile h, chunk kc.  An item's first tile
-// runs value half major (the previous item's epilogue hands O back one half
-// at a time); later tiles run sub-tile major (P buffer h is free as soon as
-// both value halves have used it).
+// sub-tile 0) -> value half dh, sub-tile h, chunk kc.  An item's first and
+// last tiles run value half major (the previous item's epilogue hands O back
+// one half at a time, and this item's epilogue starts on half 0 while half 1
+// still accumulates); the tiles between run sub-tile major (P buffer h is
+// free as soon as both value halves have used it).
 struct PvStep {
   int dh, h, kc;
 };
-__device__ __forceinline__ PvStep pv_step(int s, int nk0, int nkt, bool first_tile) {
+__device__ __forceinline__ PvStep pv_step(int s, int nk0, int nkt, bool half_major) {
   PvStep r;
   int q;
-  if (first_tile) {
+  if (half_major) {
     r.dh = s >= nkt ? 1 : 0;
     q = s - r.dh * nkt;
   } else {
@@ -536,7 +537,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int nk0 = (sub_n(n, 0) + 63) >> 6;
             const int nkt = nk0 + ((sub_n(n, 1) + 63) >> 6);
             for (int s = 0; s < 2 * nkt && ok; ++s) {
-              const PvStep q = pv_step(s, nk0, nkt, j == 0);
+              const PvStep q = pv_step(s, nk0, nkt, j == 0 || j == x.ntiles - 1);
               const int key = 128 * q.h + 64 * q.kc;
               ok = stage_load(comp ? &maps.cv4 : &maps.v4, comp ? j * kKT + key : x.t0 - 127 + key,
                               4 * q.dh, x.b);
@@ -655,12 +656,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int nk0 = (sub_n(n, 0) + 63) >> 6, nk1 = (sub_n(n, 1) + 63) >> 6;
             const int nkt = nk0 + nk1;
             for (int s = 0; s < 2 * nkt && ok; ++s) {
-              const PvStep q = pv_step(s, nk0, nkt, j == 0);
+              const bool last = j == x.ntiles - 1;
+              const PvStep q = pv_step(s, nk0, nkt, j == 0 || last);
               if (j == 0 && (s == 0 || s == nkt))  // this half of the last item's O is read out
                 ok = mbar_wait(bar(OFREE + q.dh), (nitem & 1) ^ 1, abort_flag, kWaitLimitNs, 152);
               if (q.dh == 0 && q.kc == 0) p_full(q.h);
               if (ok) chunk(q.dh, q.h, q.kc);
               if (ok && q.dh == 1 && q.kc == (q.h ? nk1 : nk0) - 1) p_done(q.h);
+              if (ok && last && s == nkt - 1) umma_commit(bar(OFULL + 0));  // O half 0 final
             }
             if (ok && nk1 == 0) {  // empty sub-tile 1: its buffer handshake still runs
               p_full(1);
@@ -670,7 +673,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             umma_commit(bar(PVDONE + (sj & 1)));   // all of tile sj's P.V
           }
           if (!ok) break;
-          umma_commit(bar(OFULL));
+          umma_commit(bar(OFULL + 1));
           u += 4;  // g stages, consumed by the epilogue
         }
         umma_commit(bar(DRAIN));
@@ -728,7 +731,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         // ---------------------------------------------------------- epilogue
-        if (!mbar_wait_warp(bar(OFULL), nitem & 1, abort_flag, kWaitLimitNs, 162) ||
+        if (!mbar_wait_warp(bar(OFULL + 0), nitem & 1, abort_flag, kWaitLimitNs, 162) ||
             !mbar_wait_cluster_warp(bar(STATSFULL), nitem & 1, abort_flag, kWaitLimitNs, 163)) {
           ok = false;
           break;
@@ -747,6 +750,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const int e = half + 2 * ee;          // g / out stage: value columns [128e, 128e + 128)
           const uint32_t ug = gbase + e;
           const uint32_t st = ug % kVStages;
+          if (ee == 1) {  // O half 1 is final once the item's last P.V completed
+            if (!mbar_wait_warp(bar(OFULL + 1), nitem & 1, abort_flag, kWaitLimitNs, 165)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
           if (!mbar_wait_warp(bar(VFULL + st), (ug / kVStages) & 1, abort_flag, kWaitLimitNs, 164)) {
             ok = false;
             break;
