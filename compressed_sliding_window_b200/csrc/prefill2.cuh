@@ -635,14 +635,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               ++u;
               if (!ok) return;
               tc_fence_after();
-              const uint32_t pa = sb + O_P + h * kPBuf;
-              const uint32_t va = sb + O_VRING + st * kVStage;
-#pragma unroll 1
-              for (int ks = 0; ks < ksteps; ++ks) {
-                const bool first = (j == 0 && h == 0 && kc == 0 && ks == 0);
-                umma_bf16(tmem + 256 * dh, sdesc_noswz(pa + kc * 16384 + 4096 * ks, 2048, 128),
-                          sdesc_sw128(va + 2048 * ks, 8192, 1024), idesc, first ? 0u : 1u);
-              }
+              // descriptors of the chunk's first K step; later steps only move
+              // the start address (bits 0-13 hold address >> 4, no carry)
+              const uint64_t ad = sdesc_noswz(sb + O_P + h * kPBuf + kc * 16384, 2048, 128);
+              const uint64_t bd = sdesc_sw128(sb + O_VRING + st * kVStage, 8192, 1024);
+              const uint32_t dt = tmem + 256 * dh;
+              const uint32_t acc0 = (j == 0 && h == 0 && kc == 0) ? 0u : 1u;
+              umma_bf16(dt, ad, bd, idesc, acc0);
+#pragma unroll
+              for (int ks = 1; ks < 4; ++ks)
+                if (ks < ksteps) umma_bf16(dt, ad + 256 * ks, bd + 128 * ks, idesc, 1u);
               umma_commit(bar(VEMPTY + st));
             };
             auto p_full = [&](int h) {
