@@ -108,17 +108,19 @@ def test_decode_bad_device_length_is_reported_not_faulted():
     assert hca.device_error()[0] == 0  # cleared
 
 
-def test_decode_many_sequences_planned_by_plan_kernel():
-    """More sequences than one CTA plans for itself: the tile prefix then comes
-    from the separate plan kernel."""
+@pytest.mark.parametrize("S", [1024, 1025, 1100])
+def test_decode_many_sequences_planned_by_plan_kernel(S):
+    """Up to 1024 sequences each CTA plans for itself (the prefix in shared
+    memory at its largest at S = 1024); above that the tile prefix comes from
+    the separate plan kernel."""
     need_gpu()
-    rng = np.random.default_rng(11)
-    lens = [int(x) for x in rng.integers(1, 700, size=1100)]
+    rng = np.random.default_rng(11 + S)
+    lens = [int(x) for x in rng.integers(1, 700, size=S)]
     max_nc = 4
     q, g, ck, cv, wk, wv = _direct_case(lens, max_nc, seed=12)
     out = _run(q, g, ck, cv, wk, wv, lens)
     ref = O.decode_forward(to64(q), to64(ck), to64(cv), to64(wk), to64(wv), lens, to64(g))
-    assert_close_out(to64(out), ref, "S=1100")
+    assert_close_out(to64(out), ref, f"S={S}")
 
 
 def test_decode_workspace_reused_across_calls_and_sizes():
