@@ -33,14 +33,18 @@
 // brings 4 (V) or 2 (g) 64-wide column slabs, already in the layout the MMA
 // and the epilogue read.
 //
-// Warp roles (416 threads): warps 0-1 TMA producers, warp 2 MMA issuer and
+// Warp roles (544 threads): warps 0-1 TMA producers, warp 2 MMA issuer and
 // TMEM owner, warps 3-10 compute: two warps per TMEM lane quadrant, so a tile
 // row is shared by two threads.  On rank 0 each of them owns one 128-key half
 // of the score tile (= one P sub-tile; the row max is exchanged through shared
 // memory under a 64-thread named barrier); on rank 1 they rescale O (each 256
-// of the 512 value columns) and run the epilogue (128 columns per stage).
-// Rank 1 also has warp 11, the P copier, and warp 12, which stores the
-// epilogue's output stages and hands them back to the producers.
+// of the 512 value columns) and run the epilogue of O's value half 0 (128
+// columns per warp).  Rank 1 also has warp 11, the P copier, warp 12, which
+// stores the epilogue's output stages and hands them back to the producers,
+// and warps 13-16, one per lane quadrant, which run the epilogue of value
+// half 1 (both of its stages) in parallel with half 0 (the epilogue is bound
+// by instruction latency, not issue slots).  Warps 11-16 of rank 0 have no
+// role.
 //
 // Code size.  The kernel is bound by instruction fetch long before its loops
 // are: every role's hot loop is kept small (32-column chunks, one code path
@@ -56,7 +60,7 @@ constexpr int kRows = 128;
 constexpr int kHeads = 64;
 constexpr int kKT = 256;     // compressed key tile
 constexpr int kWinN = 144;   // raw key tile
-constexpr int kThreads = 416;
+constexpr int kThreads = 544;
 constexpr int kScratchPerPair = 4 * 32768;   // 2 tile parities x 2 sub-tiles
 constexpr float kTau = 8.0f;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
@@ -224,12 +228,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int i = 0; i < NBAR; ++i) mbar_init(bar(i), 1);
     mbar_init(bar(SFREE + 0), 8);
     mbar_init(bar(SFREE + 1), 8);
-    mbar_init(bar(STATSFREE), 8);
+    mbar_init(bar(STATSFREE), 12);
     for (int q = 0; q < 4; ++q) mbar_init(bar(PREADY + q), 4);
     mbar_init(bar(CORR + 0), 8);
     mbar_init(bar(CORR + 1), 8);
     mbar_init(bar(OFREE + 0), 8);
-    mbar_init(bar(OFREE + 1), 8);
+    mbar_init(bar(OFREE + 1), 4);
     mbar_init(bar(STATSFULL), 4);
     for (int e = 0; e < 4; ++e) mbar_init(bar(STAGED + e), 128);
     *abort_flag = 0;
@@ -683,8 +687,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
     } else {
       // --------------------------------------------------------- correction + epilogue
+      // warps 3-10: correction, and the epilogue of value half 0 (stage half);
+      // warps 13-16 (helpers): the epilogue of value half 1 (stages 2 and 3)
+      const bool helper = warp >= 13;
       const int wq = warp & 3;
-      const int half = (warp - 3) >> 2;
+      const int half = helper ? 0 : (warp - 3) >> 2;
       const int row = wq * 32 + lane;
       const uint32_t tq = tmem + (static_cast<uint32_t>(wq * 32) << 16);
       const uint32_t tl = tq + 256 * half;     // rescale: value columns [256 half, +256)
@@ -697,7 +704,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int it = pair; it < p.items && ok; it += npairs, ++nitem) {
         const Item x = decode_item(p, it);
         ++sj;  // the first tile of an item needs no correction (its running max starts there)
-        for (int j = 1; j < x.ntiles; ++j, ++sj, ++ncorr) {
+        for (int j = 1; j < x.ntiles && !helper; ++j, ++sj, ++ncorr) {
           if (!mbar_wait_cluster_warp(bar(PREADY + (sj & 1) * 2), (sj >> 1) & 1, abort_flag,
                                       kWaitLimitNs, 160)) {
             ok = false;
@@ -733,32 +740,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         // ---------------------------------------------------------- epilogue
-        if (!mbar_wait_warp(bar(OFULL + 0), nitem & 1, abort_flag, kWaitLimitNs, 162) ||
-            !mbar_wait_cluster_warp(bar(STATSFULL), nitem & 1, abort_flag, kWaitLimitNs, 163)) {
+        // 1/l first (the S-CTA reuses its slot once all 12 warps took it),
+        // then this warp's value half of O once its last P.V completed
+        const int ee = helper ? 1 : 0;
+        if (!mbar_wait_cluster_warp(bar(STATSFULL), nitem & 1, abort_flag, kWaitLimitNs, 163)) {
           ok = false;
           break;
         }
-        tc_fence_after();
         const float il = invl_s[row];
         const float hil = 0.5f * il;
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(peerStatsFree);
+        if (!mbar_wait_warp(bar(OFULL + ee), nitem & 1, abort_flag, kWaitLimitNs, 162)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
         const uint32_t gbase = ubase + v_uses(x);
         ubase = gbase + 4;
-        // value half ee first (both warps of a quadrant, 128 columns each), so
-        // O half 0 is released to the next item halfway through
 #pragma unroll 1
-        for (int ee = 0; ee < 2; ++ee) {
-          const int e = half + 2 * ee;          // g / out stage: value columns [128e, 128e + 128)
+        for (int e2 = 0; e2 < (helper ? 2 : 1); ++e2) {
+          const int e = helper ? 2 + e2 : half;  // g / out stage: value columns [128e, 128e + 128)
           const uint32_t ug = gbase + e;
           const uint32_t st = ug % kVStages;
-          if (ee == 1) {  // O half 1 is final once the item's last P.V completed
-            if (!mbar_wait_warp(bar(OFULL + 1), nitem & 1, abort_flag, kWaitLimitNs, 165)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-          }
           if (!mbar_wait_warp(bar(VFULL + st), (ug / kVStages) & 1, abort_flag, kWaitLimitNs, 164)) {
             ok = false;
             break;
@@ -772,7 +776,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             uint32_t o[32];
             tmem_ld32(tq + 128 * e + 32 * q32, o);
             tmem_wait_ld_dep32(o);
-            if (q32 == 3) {
+            if (q32 == 3 && e2 == (helper ? 1 : 0)) {  // this warp's part of O read out
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive(bar(OFREE + ee));
