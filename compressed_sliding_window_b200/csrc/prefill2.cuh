@@ -621,61 +621,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         uint32_t u = 0, sj = 0, nitem = 0, ncorr = 0;
         bool ok = true;
         const uint32_t idesc = idesc_bf16_f32(kRows, 256, false, true);
+        // The issuing thread's time goes to its own branches as much as to
+        // waiting: the step loop is kept straight (commits and the short last
+        // K steps predicated, the ok flag checked per tile; after a failed
+        // bounded wait the abort flag makes every later wait return at once).
         for (int it = pair; it < p.items && ok; it += npairs, ++nitem) {
           const Item x = decode_item(p, it);
           for (int j = 0; j < x.ntiles && ok; ++j, ++sj) {
             const int n = tile_n(x, j);
-            if (j > 0) {  // an item's first tile never needs a rescale of O
-              ok = mbar_wait(bar(CORR + (ncorr & 1)), (ncorr >> 1) & 1, abort_flag, kWaitLimitNs,
-                             151);
-              ++ncorr;
-            }
-            // P.V of one 64-key chunk into one value half
-            auto chunk = [&](int dh, int h, int kc) {
-              const int nh = sub_n(n, h);
-              const int ksteps = min(4, (nh - 64 * kc) >> 4);
+            if (j > 0)  // an item's first tile never needs a rescale of O
+              ok &= mbar_wait(bar(CORR + (ncorr & 1)), (ncorr >> 1) & 1, abort_flag, kWaitLimitNs,
+                              151);
+            ncorr += (j > 0);
+            const bool first = j == 0, last = j == x.ntiles - 1;
+            const int nk0 = (sub_n(n, 0) + 63) >> 6, nk1 = (sub_n(n, 1) + 63) >> 6;
+            const int nkt = nk0 + nk1;
+            const uint32_t pfree0 = bar(PFREE + (sj & 1) * 2);
+#pragma unroll 1
+            for (int s = 0; s < 2 * nkt; ++s) {
+              const PvStep q = pv_step(s, nk0, nkt, first || last);
+              if (first && (s == 0 || s == nkt))  // this half of the last item's O is read out
+                ok &= mbar_wait(bar(OFREE + q.dh), (nitem & 1) ^ 1, abort_flag, kWaitLimitNs, 152);
+              if (q.dh == 0 && q.kc == 0)
+                ok &= mbar_wait(bar(PFULL + q.h), sj & 1, abort_flag, kWaitLimitNs, 150);
+              // P.V of one 64-key chunk into one value half
+              const int ksteps = min(4, (sub_n(n, q.h) - 64 * q.kc) >> 4);
               const uint32_t st = u % kVStages;
-              ok = mbar_wait(bar(VFULL + st), (u / kVStages) & 1, abort_flag, kWaitLimitNs, 153);
+              ok &= mbar_wait(bar(VFULL + st), (u / kVStages) & 1, abort_flag, kWaitLimitNs, 153);
               ++u;
-              if (!ok) return;
               tc_fence_after();
               // descriptors of the chunk's first K step; later steps only move
               // the start address (bits 0-13 hold address >> 4, no carry)
-              const uint64_t ad = sdesc_noswz(sb + O_P + h * kPBuf + kc * 16384, 2048, 128);
+              const uint64_t ad = sdesc_noswz(sb + O_P + q.h * kPBuf + q.kc * 16384, 2048, 128);
               const uint64_t bd = sdesc_sw128(sb + O_VRING + st * kVStage, 8192, 1024);
-              const uint32_t dt = tmem + 256 * dh;
-              const uint32_t acc0 = (j == 0 && h == 0 && kc == 0) ? 0u : 1u;
-              umma_bf16(dt, ad, bd, idesc, acc0);
-#pragma unroll
-              for (int ks = 1; ks < 4; ++ks)
-                if (ks < ksteps) umma_bf16(dt, ad + 256 * ks, bd + 128 * ks, idesc, 1u);
+              const uint32_t dt = tmem + 256 * q.dh;
+              umma_bf16(dt, ad, bd, idesc, (first && q.h == 0 && q.kc == 0) ? 0u : 1u);
+              umma_bf16_if(dt, ad + 256, bd + 128, idesc, 1u, ksteps > 1);
+              umma_bf16_if(dt, ad + 512, bd + 256, idesc, 1u, ksteps > 2);
+              umma_bf16_if(dt, ad + 768, bd + 384, idesc, 1u, ksteps > 3);
               umma_commit(bar(VEMPTY + st));
-            };
-            auto p_full = [&](int h) {
-              if (ok) ok = mbar_wait(bar(PFULL + h), sj & 1, abort_flag, kWaitLimitNs, 150);
+              // P buffer h done once value half 1 used its last chunk; O half 0
+              // final after the last tile's half-0 pass
+              const bool pdone = q.dh == 1 && q.kc == (q.h ? nk1 : nk0) - 1;
+              umma_commit_if(bar(PBUFFREE + q.h), pdone);             // smem P buffer reusable
+              umma_commit_mc_if(pfree0 + 8 * q.h, 0x1, pdone);        // scratch slot (rank 0)
+              umma_commit_if(bar(OFULL + 0), last && s == nkt - 1);
+            }
+            if (nk1 == 0) {  // empty sub-tile 1: its buffer handshake still runs
+              ok &= mbar_wait(bar(PFULL + 1), sj & 1, abort_flag, kWaitLimitNs, 150);
               tc_fence_after();
-            };
-            auto p_done = [&](int h) {
-              umma_commit(bar(PBUFFREE + h));                       // smem P buffer h reusable
-              umma_commit_mc(bar(PFREE + (sj & 1) * 2 + h), 0x1);   // scratch slot reusable (rank 0)
-            };
-            const int nk0 = (sub_n(n, 0) + 63) >> 6, nk1 = (sub_n(n, 1) + 63) >> 6;
-            const int nkt = nk0 + nk1;
-            for (int s = 0; s < 2 * nkt && ok; ++s) {
-              const bool last = j == x.ntiles - 1;
-              const PvStep q = pv_step(s, nk0, nkt, j == 0 || last);
-              if (j == 0 && (s == 0 || s == nkt))  // this half of the last item's O is read out
-                ok = mbar_wait(bar(OFREE + q.dh), (nitem & 1) ^ 1, abort_flag, kWaitLimitNs, 152);
-              if (q.dh == 0 && q.kc == 0) p_full(q.h);
-              if (ok) chunk(q.dh, q.h, q.kc);
-              if (ok && q.dh == 1 && q.kc == (q.h ? nk1 : nk0) - 1) p_done(q.h);
-              if (ok && last && s == nkt - 1) umma_commit(bar(OFULL + 0));  // O half 0 final
+              umma_commit(bar(PBUFFREE + 1));
+              umma_commit_mc(pfree0 + 8, 0x1);
             }
-            if (ok && nk1 == 0) {  // empty sub-tile 1: its buffer handshake still runs
-              p_full(1);
-              if (ok) p_done(1);
-            }
-            if (!ok) break;
             umma_commit(bar(PVDONE + (sj & 1)));   // all of tile sj's P.V
           }
           if (!ok) break;
