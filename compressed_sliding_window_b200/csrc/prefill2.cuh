@@ -304,21 +304,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int it = pair; it < p.items && ok; it += npairs, ++nitem) {
           const Item x = decode_item(p, it);
           for (int j = 0; j < x.ntiles && ok; ++j, ++sj) {
+            // straight step loop, predicated commits (see the O-CTA issuer)
             const uint32_t buf = sj & 1;
-            ok = mbar_wait(bar(SFREE + buf), ((sj >> 1) & 1) ^ 1, abort_flag, kWaitLimitNs, 120);
-            if (!ok) break;
-            tc_fence_after();
+            ok &= mbar_wait(bar(SFREE + buf), ((sj >> 1) & 1) ^ 1, abort_flag, kWaitLimitNs, 120);
             const uint32_t idesc = idesc_bf16_f32(kRows, tile_n(x, j), false, false);
             const uint32_t dS = tmem + 256 * buf;
+            const bool first = j == 0, last = j + 1 == x.ntiles;
 #pragma unroll 1
-            for (int d = 0; d < 8 && ok; ++d, ++u) {
-              if (j == 0 && (d & 3) == 0) {
-                ok = mbar_wait(bar(QFULL + (d >> 2)), nitem & 1, abort_flag, kWaitLimitNs, 121);
-                if (!ok) break;
-              }
+            for (int d = 0; d < 8; ++d, ++u) {
+              if (first && (d & 3) == 0)
+                ok &= mbar_wait(bar(QFULL + (d >> 2)), nitem & 1, abort_flag, kWaitLimitNs, 121);
               const uint32_t st = u % kKStages;
-              ok = mbar_wait(bar(KFULL + st), (u / kKStages) & 1, abort_flag, kWaitLimitNs, 122);
-              if (!ok) break;
+              ok &= mbar_wait(bar(KFULL + st), (u / kKStages) & 1, abort_flag, kWaitLimitNs, 122);
               tc_fence_after();
               const uint32_t qa = sb + S_Q + (d >> 2) * kQHalf + (d & 3) * 16384;
               const uint32_t ka = sb + S_KRING + st * kKStage;
@@ -327,9 +324,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 umma_bf16(dS, sdesc_sw128(qa + 32 * k, 16, 1024), sdesc_sw128(ka + 32 * k, 16, 1024),
                           idesc, (d | k) != 0);
               umma_commit(bar(KEMPTY + st));
-              if (j + 1 == x.ntiles && (d & 3) == 3) umma_commit(bar(QEMPTY + (d >> 2)));
+              umma_commit_if(bar(QEMPTY + (d >> 2)), last && (d & 3) == 3);
             }
-            if (!ok) break;
             umma_commit(bar(SFULL + buf));
           }
         }
