@@ -659,9 +659,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               // P buffer h done once value half 1 used its last chunk; O half 0
               // final after the last tile's half-0 pass
               const bool pdone = q.dh == 1 && q.kc == (q.h ? nk1 : nk0) - 1;
-              umma_commit_if(bar(PBUFFREE + q.h), pdone);             // smem P buffer reusable
-              umma_commit_mc_if(pfree0 + 8 * q.h, 0x1, pdone);        // scratch slot (rank 0)
-              umma_commit_if(bar(OFULL + 0), last && s == nkt - 1);
+              const bool o0 = last && s == nkt - 1;
+              if (pdone || o0) {  // rare: one branch instead of three predicated commits a step
+                umma_commit_if(bar(PBUFFREE + q.h), pdone);           // smem P buffer reusable
+                umma_commit_mc_if(pfree0 + 8 * q.h, 0x1, pdone);      // scratch slot (rank 0)
+                umma_commit_if(bar(OFULL + 0), o0);
+              }
             }
             if (nk1 == 0) {  // empty sub-tile 1: its buffer handshake still runs
               ok &= mbar_wait(bar(PFULL + 1), sj & 1, abort_flag, kWaitLimitNs, 150);
