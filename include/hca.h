@@ -114,7 +114,8 @@ size_t hca_decode_workspace_size(int S);
 
 /*
  * hca_decode — one new token per sequence (split-KV over all SMs, then a
- * log-sum-exp combine).
+ * log-sum-exp combine, in one cooperative launch of one CTA per SM; above
+ * 1024 sequences a one-CTA plan kernel runs first).
  *   For sequence i with context length L = ctx_len[i] (which counts the new
  *   token, so the query sits at t = L - 1):
  *     keys   = [ck[i, 0 : nc(L-1)] ; the min(L, 128) newest raw keys]
