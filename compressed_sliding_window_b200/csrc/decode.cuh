@@ -11,9 +11,11 @@
 // compressed tiles + one window tile).  The tiles of all sequences are laid
 // end to end and CTA c takes the contiguous range [floor(cN/G), floor((c+1)N/G)),
 // so every SM streams the same number of cache bytes whatever the length mix.
-// A CTA writes one partial (unnormalised O, running max m, running sum l) per
+// A CTA writes one partial (O / l in bf16, running max m, running sum l) per
 // sequence it touches, into slot c + i of the workspace (slots never collide:
 // a CTA's sequences are consecutive and later CTAs start at later sequences).
+// Up to kInlineSeqs sequences every CTA computes the tile prefix itself in
+// shared memory; beyond that a one-CTA plan kernel does.
 // The launch is cooperative; after every CTA has written its partials (an
 // atomic counter, bounded spin) every CTA merges a share of the (sequence,
 // head) rows, its partial rows staged in shared memory by bulk copies.
