@@ -146,19 +146,20 @@ hca_status_t hca_decode(const hca_bf16* q, const hca_bf16* ck, const hca_bf16* c
  *   latency-critical serving loop where a cudaMalloc (which can synchronise
  *   the whole device) is not allowed.  This entry point takes the same
  *   inputs and output as hca_decode but no workspace; its scratch lives in
- *   one fixed device array inside the library (224 split slots of 131,584
- *   bytes plus a small index: about 29.5 MB), which every GPU that loads the
- *   library keeps until the process exits.
+ *   one fixed device array inside the library (224 split slots of 66,048
+ *   bytes plus a small index and the grid-barrier counter: about 14.8 MB),
+ *   which every GPU that loads the library keeps until the process exits.
  *   Limits: S <= HCA_NOALLOC_MAX_SEQS (64); larger S returns
  *   HCA_ERR_UNSUPPORTED without launching.  The split uses at most
  *   HCA_NOALLOC_MAX_CTAS (160) CTAs.
  *   Set-up: the first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current) and caches it; make that
  *   first call outside any stream capture.  Nothing is allocated, ever.
- *   Sharing: every call uses the same array.  Nothing in it needs to start at
- *   zero (each call writes every scratch value it later reads), but two calls
- *   that overlap on the GPU (other streams, other threads) race on it:
- *   serialise them.
+ *   Sharing: every call uses the same array.  Its grid-barrier counter starts
+ *   at zero when the library loads and every call leaves it valid (each call
+ *   writes every other scratch value it later reads), but two calls that
+ *   overlap on the GPU (other streams, other threads) race on it: serialise
+ *   them.
  */
 #define HCA_NOALLOC_MAX_SEQS 64
 #define HCA_NOALLOC_MAX_CTAS 160
