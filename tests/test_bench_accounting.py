@@ -1,0 +1,38 @@
+"""The bench's closed-form work counts (FLOPs and bytes behind every roofline
+figure) agree with the oracle's counts and with values worked out by hand."""
+import bench
+from oracle import hca_oracle as O
+
+
+def test_nc_matches_visibility_rule():
+    # entry j is visible from position t once its whole block lies outside the
+    # window: nc(t) = max(0, floor((t - 127) / 128))
+    assert [bench.nc_of(t) for t in (0, 126, 127, 254, 255, 382, 383)] == [0, 0, 0, 0, 1, 1, 2]
+    for t in range(0, 2000, 37):
+        assert bench.nc_of(t) == O.num_visible_blocks(t)
+
+
+def test_visited_pairs_agree_with_oracle():
+    for T in (1, 127, 128, 129, 255, 256, 1000, 4096):
+        assert bench.visited_pairs(T) == O.visited_pairs(T)
+    # T = 256: every position sees min(t + 1, 128) raw keys, only t = 255
+    # also sees one compressed entry
+    assert bench.visited_pairs(256) == sum(min(t + 1, 128) for t in range(256)) + 1
+
+
+def test_prefill_bytes_32k():
+    # q, g, out: 3 x T x 64 x 512 bf16; k, v: 2 x T x 512; cK, cV: 2 x 256 x 512;
+    # s: T -- all bf16 (2 bytes)
+    T = 32768
+    by_hand = 2 * (3 * T * 64 * 512 + 2 * T * 512 + 2 * (T // 128) * 512 + T)
+    assert bench.prefill_bytes(1, T) == by_hand == 6510149632
+
+
+def test_decode_cache_keys():
+    assert bench.decode_cache_keys([1]) == 1
+    assert bench.decode_cache_keys([128]) == 128
+    assert bench.decode_cache_keys([255]) == 128
+    assert bench.decode_cache_keys([256]) == 129
+    assert bench.decode_cache_keys([131072]) == 1023 + 128
+    lens = [78841, 921936, 130194, 1, 300]
+    assert bench.decode_cache_keys(lens) == O.decode_keys(lens)
