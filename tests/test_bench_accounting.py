@@ -36,3 +36,12 @@ def test_decode_cache_keys():
     assert bench.decode_cache_keys([131072]) == 1023 + 128
     lens = [78841, 921936, 130194, 1, 300]
     assert bench.decode_cache_keys(lens) == O.decode_keys(lens)
+
+
+def test_flops_per_pair():
+    # per visited (query, key) pair and head: q.k (512 multiply-adds) and
+    # p.v (512 multiply-adds), 2 FLOPs each, 64 heads
+    assert bench.FLOP_PER_PAIR == 64 * (2 * 512 + 2 * 512)
+    # the two prefill workloads' totals quoted beside the bench numbers
+    assert round(bench.visited_pairs(32768) * bench.FLOP_PER_PAIR / 1e12, 3) == 1.092
+    assert round(bench.visited_pairs(131072) * bench.FLOP_PER_PAIR / 1e13, 3) == 1.097
