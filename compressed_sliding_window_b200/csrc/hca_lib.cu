@@ -75,12 +75,19 @@ bool make_map4(CUtensorMap* m, const void* base, uint64_t Y, uint64_t W, uint32_
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// How many 2-CTA clusters of the prefill kernel fit on the device at once.
+constexpr int kMaxDevices = 64;
+
+// How many 2-CTA clusters of the prefill kernel fit on the current device at
+// once.  The shared-memory attribute is a per-device property of the kernel,
+// so it is set, and the occupancy asked, once for every device the process
+// uses (with that device current).
 int prefill_max_pairs() {
-  static int cached = -1;
+  static int cached[kMaxDevices] = {};
   static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
   std::lock_guard<std::mutex> lock(mu);
-  if (cached > 0) return cached;
+  if (cached[dev] > 0) return cached[dev];
   namespace P = hca::prefill2;
   if (cudaFuncSetAttribute(P::prefill2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            P::kSmemAlloc) != cudaSuccess)
@@ -99,8 +106,8 @@ int prefill_max_pairs() {
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, P::prefill2_kernel, &cfg) != cudaSuccess || n <= 0)
     return -1;
-  cached = n;
-  return cached;
+  cached[dev] = n;
+  return n;
 }
 
 // The decode pass: for more than kInlineSeqs sequences the plan kernel first
@@ -323,22 +330,16 @@ constexpr size_t kNoAllocScratchBytes =
 // kNoAllocSlots split slots, then the tile prefix.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mutex;
-void* g_noalloc_addr[kMaxDevices] = {};
-
-// Device address of g_noalloc_scratch on the current device (looked up once
-// per device, with that device current).  Null on failure.
+// Device address of g_noalloc_scratch in the current device's context.  The
+// array's name is only a host-side handle, so the address is asked of the
+// runtime, with the device current.  It is asked on every call rather than
+// cached: a cached address would outlive a cudaDeviceReset (which unloads the
+// module and places the array anew in the next context).  The first call on a
+// device loads the module there.  Null on failure.
 void* noalloc_scratch_address() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (g_noalloc_addr[dev] == nullptr) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
-    g_noalloc_addr[dev] = ptr;
-  }
-  return g_noalloc_addr[dev];
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+  return ptr;
 }
 
 }  // namespace

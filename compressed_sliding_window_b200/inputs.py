@@ -84,6 +84,16 @@ def normal_bf16(base: int, name: str, rows: int, row_shape: Sequence[int] = (),
     return out
 
 
+def chunk_rows(base: int, name: str, c: int, rows: int, row_shape: Sequence[int] = (),
+               scale: float = 1.0) -> torch.Tensor:
+    """Rows [c * CHUNK, min(rows, (c + 1) * CHUNK)) of the tensor that
+    ``normal_bf16(base, name, rows, row_shape, scale)`` draws, without drawing
+    the rest (same generator, same values)."""
+    r0 = c * CHUNK
+    r1 = min(rows, r0 + CHUNK)
+    return _draw_chunk(base, name, c, r1 - r0, tuple(row_shape), scale)
+
+
 # ---------------------------------------------------------------------------
 # Workload definitions
 # ---------------------------------------------------------------------------
@@ -182,20 +192,3 @@ def decode_query(cfg: DecodeConfig):
     q = normal_bf16(base, "q", cfg.S, (HEADS, HEAD_DIM))
     g = normal_bf16(base, "g", cfg.S, (HEADS, HEAD_DIM))
     return q, g
-
-
-def sample_positions(T: int, blk: int = BLOCK) -> List[int]:
-    """Deterministic row sample for large prefill parity checks: every row of
-    query blocks 0, 1, 2 and of the last three blocks, plus rows r in
-    {0, 1, 126, 127} of every block, plus the last position."""
-    nblk = (T + blk - 1) // blk
-    pos = set()
-    for j in list(range(min(3, nblk))) + list(range(max(0, nblk - 3), nblk)):
-        pos.update(range(j * blk, min(T, (j + 1) * blk)))
-    for j in range(nblk):
-        for r in (0, 1, blk - 2, blk - 1):
-            t = j * blk + r
-            if t < T:
-                pos.add(t)
-    pos.add(T - 1)
-    return sorted(pos)

@@ -74,8 +74,10 @@ hca_status_t hca_compress(const hca_bf16* k, const hca_bf16* v, const hca_bf16* 
 
 /*
  * hca_prefill_workspace_size — bytes of device scratch hca_prefill_fwd needs
- * on the current device (probability tiles in flight between the two CTAs of
- * each cluster; about 128 KB per cluster, under 10 MB on a B200).
+ * on the current device (probability tiles in flight between the CTAs of
+ * each cluster; under 10 MB on a B200).  The answer depends on how many
+ * clusters fit on the device, which is queried once per device.  Returns 0
+ * for B < 1 or T < 1 or when the query fails.
  */
 size_t hca_prefill_workspace_size(int B, int T);
 
@@ -152,9 +154,11 @@ hca_status_t hca_decode(const hca_bf16* q, const hca_bf16* ck, const hca_bf16* c
  *   Limits: S <= HCA_NOALLOC_MAX_SEQS (64); larger S returns
  *   HCA_ERR_UNSUPPORTED without launching.  The split uses at most
  *   HCA_NOALLOC_MAX_CTAS (160) CTAs.
- *   Set-up: the first call on a device looks up the array's device address
- *   (cudaGetSymbolAddress, with that device current) and caches it; make that
- *   first call outside any stream capture.  Nothing is allocated, ever.
+ *   Set-up: every call looks up the array's device address in the current
+ *   device's context (cudaGetSymbolAddress, with that device current; the
+ *   array's name in host code is only a handle).  The first call on a device
+ *   also loads the library's module there, so make that first call outside
+ *   any stream capture.  Nothing is allocated, ever.
  *   Sharing: every call uses the same array.  Its grid-barrier counter starts
  *   at zero when the library loads and every call leaves it valid (each call
  *   writes every other scratch value it later reads), but two calls that
@@ -173,6 +177,12 @@ hca_status_t hca_decode_noalloc(const hca_bf16* q, const hca_bf16* ck, const hca
  * device-side error word of the current device.  Returns HCA_OK,
  * HCA_ERR_TIMEOUT, HCA_ERR_DEVICE_INPUT or HCA_ERR_CUDA.  `where`, if not
  * NULL, receives an internal code naming the wait that gave up.
+ * The error word is one per device for the whole process: every stream and
+ * every host thread that launches this library's kernels on that device
+ * records into it, and this call reads and clears it for all of them.  A
+ * caller that drives one device from several threads or streams therefore
+ * sees (and clears) errors of the others' launches too; serialise the checks
+ * or attribute errors per device, not per stream.
  */
 hca_status_t hca_get_device_error(hca_stream_t stream, unsigned int* where);
 

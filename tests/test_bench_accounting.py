@@ -45,3 +45,11 @@ def test_flops_per_pair():
     # the two prefill workloads' totals quoted beside the bench numbers
     assert round(bench.visited_pairs(32768) * bench.FLOP_PER_PAIR / 1e12, 3) == 1.092
     assert round(bench.visited_pairs(131072) * bench.FLOP_PER_PAIR / 1e13, 3) == 1.097
+
+
+def test_compress_bytes():
+    # per complete block: K and V rows (2 x 128 x 512 bf16), the 128 scores,
+    # and the two 512-wide entries written
+    assert bench.compress_bytes(1, 131072) == 1024 * (2 * 128 * 512 * 2 + 128 * 2 + 2 * 512 * 2)
+    assert bench.compress_bytes(1, 131072) == 1024 * 264448
+    assert bench.compress_bytes(2, 300) == 2 * 2 * 264448    # the ragged tail is not read
