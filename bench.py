@@ -425,7 +425,7 @@ def run_ours(args):
     value = job_throughput(flops, world, args.steps, max_ms) / 1e12
     tflops_kernel = flops / (prefill_ms / 1e3) / 1e12
     alg_bytes = prefill_bytes(B, T)
-    traffic = read_traffic("prefill2.cuh", "prefill2_T131072_traffic.txt")
+    traffic = read_traffic("prefill3.cuh", "prefill3_T131072_traffic.txt")
     c_bytes = compress_bytes(B, T)
     result = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
@@ -437,7 +437,7 @@ def run_ours(args):
                                "gate fused",
                    "global_batch": world * B, "seq_len": T, "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2 (17.5 GB read, 8.6 GB written per step)"},
-        "roofline": {"kernel": "prefill2_kernel", "bound": "tensor", "achieved": tflops_kernel,
+        "roofline": {"kernel": "prefill3_kernel", "bound": "tensor", "achieved": tflops_kernel,
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": tflops_kernel / peaks["bf16_tflops"],
                      "peak_source": peaks["source"] + " (bf16 dense, burst)",
@@ -541,10 +541,10 @@ def bench_prefill_side(cfg, dev, peaks, args):
                        + (f" (K x{cfg.k_scale})" if cfg.k_scale != 1.0 else ""),
            "tflops": flops / (step_ms / 1e3) / 1e12, "ms_per_step": step_ms,
            "prefill_ms_per_launch": ms, "flops": flops, "algorithmic_bytes": alg,
-           "roofline": {"kernel": "prefill2_kernel", "bound": "hbm", "achieved": gbs,
+           "roofline": {"kernel": "prefill3_kernel", "bound": "hbm", "achieved": gbs,
                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
                         "peak_source": peaks["source"],
-                        "traffic": read_traffic("prefill2.cuh", "prefill2_T32768_traffic.txt"),
+                        "traffic": read_traffic("prefill3.cuh", "prefill3_T32768_traffic.txt"),
                         "tensor": {"achieved": tf, "peak": peaks["bf16_tflops"],
                                    "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"]}}}
     del d, out, ck, cv, ws
@@ -637,6 +637,16 @@ def run_profile_case(args):
         q, gg, k, v, s = rnd(1, T, 64, 512), rnd(1, T, 64, 512), rnd(1, T, 512, s=0.5), rnd(1, T, 512), rnd(1, T)
         for _ in range(args.warmup):
             hca.forward(q, k, v, s, gg)
+    elif kind == "decode-long":
+        # the 16-sequence long-context workload's lengths, cache drawn on the device
+        from compressed_sliding_window_b200 import inputs as I
+        lens = I.decode_ctx_lens(I.DECODE_16xLONG)
+        S, nc = len(lens), 8191
+        ck, cv = rnd(S, nc, 512), rnd(S, nc, 512)
+        wk, wv, q, gg = rnd(S, 128, 512), rnd(S, 128, 512), rnd(S, 64, 512), rnd(S, 64, 512)
+        ctx = torch.tensor(lens, dtype=torch.int32, device=dev)
+        for _ in range(args.warmup):
+            hca.decode(q, ck, cv, wk, wv, ctx, gg)
     elif kind == "decode":
         S, L = int(dims[0]), int(dims[1])
         nc = L // 128
@@ -717,7 +727,7 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=50)
     ap.add_argument("--side-steps", type=int, default=20)
     ap.add_argument("--profile-case", default=None,
-                    help="prefill:T or decode:S:L -- a few untimed launches for ncu")
+                    help="prefill:T, decode:S:L or decode-long -- a few untimed launches for ncu")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     if args.profile_case:

@@ -15,7 +15,7 @@
 #include "../../include/hca.h"
 #include "hca_ptx.cuh"
 #include "compress.cuh"
-#include "prefill2.cuh"
+#include "prefill3.cuh"
 #include "decode.cuh"
 
 namespace {
@@ -77,34 +77,48 @@ bool make_map4(CUtensorMap* m, const void* base, uint64_t Y, uint64_t W, uint32_
 
 constexpr int kMaxDevices = 64;
 
-// How many 2-CTA clusters of the prefill kernel fit on the current device at
+// 2-D byte view [rows][256] of a buffer, box (256, box_rows), no swizzle:
+// moves contiguous 256-byte rows.
+bool make_map_bytes(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {256, rows};
+  const cuuint64_t strides[1] = {256};
+  const cuuint32_t box[2] = {256, box_rows};
+  const cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// How many 4-CTA clusters of the prefill kernel fit on the current device at
 // once.  The shared-memory attribute is a per-device property of the kernel,
 // so it is set, and the occupancy asked, once for every device the process
 // uses (with that device current).
-int prefill_max_pairs() {
+int prefill_max_clusters() {
   static int cached[kMaxDevices] = {};
   static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
   std::lock_guard<std::mutex> lock(mu);
   if (cached[dev] > 0) return cached[dev];
-  namespace P = hca::prefill2;
-  if (cudaFuncSetAttribute(P::prefill2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  namespace P = hca::prefill3;
+  if (cudaFuncSetAttribute(P::prefill3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            P::kSmemAlloc) != cudaSuccess)
     return -1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2, 1, 1);
+  cfg.gridDim = dim3(4, 1, 1);
   cfg.blockDim = dim3(P::kThreads, 1, 1);
   cfg.dynamicSmemBytes = P::kSmemAlloc;
   cudaLaunchAttribute attr;
   attr.id = cudaLaunchAttributeClusterDimension;
-  attr.val.clusterDim.x = 2;
+  attr.val.clusterDim.x = 4;
   attr.val.clusterDim.y = 1;
   attr.val.clusterDim.z = 1;
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, P::prefill2_kernel, &cfg) != cudaSuccess || n <= 0)
+  if (cudaOccupancyMaxActiveClusters(&n, P::prefill3_kernel, &cfg) != cudaSuccess || n <= 0)
     return -1;
   cached[dev] = n;
   return n;
@@ -187,18 +201,18 @@ hca_status_t hca_compress(const hca_bf16* k, const hca_bf16* v, const hca_bf16* 
 
 size_t hca_prefill_workspace_size(int B, int T) {
   if (B < 1 || T < 1) return 0;
-  const long long items = static_cast<long long>(B) * ((T + 1) / 2);
-  const int max_pairs = prefill_max_pairs();
-  if (max_pairs <= 0) return 0;
-  const long long pairs = items < max_pairs ? items : max_pairs;
-  return static_cast<size_t>(pairs) * hca::prefill2::kScratchPerPair + 256;
+  const long long items = static_cast<long long>(B) * ((T + 3) / 4);
+  const int max_clusters = prefill_max_clusters();
+  if (max_clusters <= 0) return 0;
+  const long long clusters = items < max_clusters ? items : max_clusters;
+  return static_cast<size_t>(clusters) * hca::prefill3::kScratchPerCluster + 256;
 }
 
 hca_status_t hca_prefill_fwd(const hca_bf16* q, const hca_bf16* k, const hca_bf16* v,
                              const hca_bf16* ck, const hca_bf16* cv, const hca_bf16* g, int B,
                              int T, int H, float scale, hca_bf16* out, float* lse, void* ws,
                              size_t ws_bytes, hca_stream_t stream) {
-  namespace P = hca::prefill2;
+  namespace P = hca::prefill3;
   if (H != HCA_NUM_HEADS) return HCA_ERR_UNSUPPORTED;
   if (B < 1 || T < 1 || !scale_ok(scale)) return HCA_ERR_INVALID_ARG;
   if (q == nullptr || k == nullptr || v == nullptr || g == nullptr || out == nullptr ||
@@ -211,24 +225,27 @@ hca_status_t hca_prefill_fwd(const hca_bf16* q, const hca_bf16* k, const hca_bf1
   for (const void* ptr : ptrs)
     if (ptr != nullptr && !aligned16(ptr)) return HCA_ERR_INVALID_ARG;
   if (static_cast<long long>(T) * HCA_NUM_HEADS > 0x7fffffffLL) return HCA_ERR_UNSUPPORTED;
-  const long long row_tiles = (T + 1) / 2;
-  const long long items = static_cast<long long>(B) * row_tiles * 2;
+  const long long row_tiles = (T + 3) / 4;
+  const long long items = static_cast<long long>(B) * row_tiles;
   if (items > 0x7fffffffLL) return HCA_ERR_UNSUPPORTED;
 
-  const long long items2 = static_cast<long long>(B) * row_tiles;
-  if (items2 > 0x7fffffffLL) return HCA_ERR_UNSUPPORTED;
-  (void)items;
+  const int max_clusters = prefill_max_clusters();
+  if (max_clusters <= 0) return HCA_ERR_CUDA;
+  const int clusters = static_cast<int>(items < max_clusters ? items : max_clusters);
+  if (ws_bytes < static_cast<size_t>(clusters) * P::kScratchPerCluster) return HCA_ERR_INVALID_ARG;
 
   P::Maps maps;
   const uint64_t rows = static_cast<uint64_t>(T) * HCA_NUM_HEADS;
+  const uint64_t prows = static_cast<uint64_t>(clusters) * P::kScratchPerCluster / 256;
   bool ok = make_map4(&maps.q4, q, rows, B, 128, 4) && make_map4(&maps.g4, g, rows, B, 128, 2) &&
             make_map4(&maps.out4, out, rows, B, 128, 2) &&
-            make_map(&maps.kwin, k, HCA_HEAD_DIM, T, B, P::kWinN) &&
-            make_map4(&maps.v4, v, T, B, 64, 4);
+            make_map(&maps.kwin, k, HCA_HEAD_DIM, T, B, P::kWinHalf) &&
+            make_map4(&maps.v4, v, T, B, 128, 2) && make_map4(&maps.v4t, v, T, B, 16, 1) &&
+            make_map_bytes(&maps.p128, ws, prows, 128) && make_map_bytes(&maps.p16, ws, prows, 16);
   if (ok && nb > 0) {
-    ok = make_map(&maps.ck, ck, HCA_HEAD_DIM, nb, B, 64) && make_map4(&maps.cv4, cv, nb, B, 64, 4);
+    ok = make_map(&maps.ck, ck, HCA_HEAD_DIM, nb, B, 64) && make_map4(&maps.cv4, cv, nb, B, 128, 2);
   } else if (ok) {  // no compressed entry exists; these maps are never used
-    ok = make_map(&maps.ck, k, HCA_HEAD_DIM, T, B, 64) && make_map4(&maps.cv4, v, T, B, 64, 4);
+    ok = make_map(&maps.ck, k, HCA_HEAD_DIM, T, B, 64) && make_map4(&maps.cv4, v, T, B, 128, 2);
   }
   if (!ok) return HCA_ERR_CUDA;
 
@@ -236,15 +253,11 @@ hca_status_t hca_prefill_fwd(const hca_bf16* q, const hca_bf16* k, const hca_bf1
   prm.B = B;
   prm.T = T;
   prm.row_tiles = static_cast<int>(row_tiles);
-  prm.items = static_cast<int>(items2);
+  prm.items = static_cast<int>(items);
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.lse = lse;
   prm.pscratch = static_cast<uint8_t*>(ws);
-  const int max_pairs = prefill_max_pairs();
-  if (max_pairs <= 0) return HCA_ERR_CUDA;
-  const int pairs = static_cast<int>(items2 < max_pairs ? items2 : max_pairs);
-  if (ws_bytes < static_cast<size_t>(pairs) * P::kScratchPerPair) return HCA_ERR_INVALID_ARG;
-  P::prefill2_kernel<<<2 * pairs, P::kThreads, P::kSmemAlloc, stream>>>(maps, prm);
+  P::prefill3_kernel<<<4 * clusters, P::kThreads, P::kSmemAlloc, stream>>>(maps, prm);
   return launch_status();
 }
 
