@@ -54,13 +54,16 @@ def lib() -> ctypes.CDLL:
         L.hca_decode_workspace_size.argtypes = [i]
         L.hca_decode_workspace_size.restype = sz
         L.hca_decode.argtypes = [vp, vp, vp, i, vp, vp, vp, vp, i, i, f, vp, sz, vp, vp]
+        L.hca_cache_append.argtypes = [vp, vp, vp, vp, i, vp, vp, vp, vp, vp, i, vp]
+        L.hca_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i, i, f, vp, vp, vp, vp, vp, i, vp,
+                                      sz, vp, vp]
         L.hca_get_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
         L.hca_selftest_bounded_wait.argtypes = [i, vp]
         L.hca_status_string.argtypes = [i]
         L.hca_status_string.restype = ctypes.c_char_p
         L.hca_version.restype = i
         for name in ("hca_compress", "hca_prefill_fwd", "hca_decode", "hca_get_device_error",
-                     "hca_selftest_bounded_wait"):
+                     "hca_selftest_bounded_wait", "hca_cache_append", "hca_decode_step"):
             getattr(L, name).restype = i
         _LIB = L
     return _LIB
@@ -198,6 +201,63 @@ def decode(q: torch.Tensor, ck: torch.Tensor, cv: torch.Tensor, wk: torch.Tensor
         wk.data_ptr(), wv.data_ptr(), ctx_len.data_ptr(), g.data_ptr(), S, H,
         ctypes.c_float(scale), workspace.data_ptr(), workspace.numel(), out.data_ptr(),
         _stream(q.device)))
+    return out
+
+
+def _check_append(k_new, v_new, s_new, ctx_len, wk, wv, ws, ck, cv):
+    S = k_new.shape[0]
+    _check(k_new, "k_new", (S, HEAD_DIM))
+    _check(v_new, "v_new", (S, HEAD_DIM))
+    _check(s_new, "s_new", (S,))
+    _check(ctx_len, "ctx_len", (S,), dtype=torch.int32)
+    _check(wk, "wk", (S, WINDOW, HEAD_DIM))
+    _check(wv, "wv", (S, WINDOW, HEAD_DIM))
+    _check(ws, "ws", (S, WINDOW))
+    max_nc = ck.shape[1]
+    _check(ck, "ck", (S, max_nc, HEAD_DIM))
+    _check(cv, "cv", (S, max_nc, HEAD_DIM))
+    return S, max_nc
+
+
+def cache_append(k_new: torch.Tensor, v_new: torch.Tensor, s_new: torch.Tensor,
+                 ctx_len: torch.Tensor, wk: torch.Tensor, wv: torch.Tensor, ws: torch.Tensor,
+                 ck: torch.Tensor, cv: torch.Tensor) -> None:
+    """Append one token per sequence to the decode cache, in place.
+
+    k_new, v_new [S, 512]; s_new [S]; ctx_len [S] int32 (counts the new
+    token); wk, wv [S, 128, 512] and ws [S, 128] rings (slot = position mod
+    128); ck, cv [S, max_nc, 512]: entry L/128 - 1 is written when L is a
+    multiple of 128."""
+    S, max_nc = _check_append(k_new, v_new, s_new, ctx_len, wk, wv, ws, ck, cv)
+    _ok("hca_cache_append", lib().hca_cache_append(
+        k_new.data_ptr(), v_new.data_ptr(), s_new.data_ptr(), ctx_len.data_ptr(), S,
+        wk.data_ptr(), wv.data_ptr(), ws.data_ptr(), _ptr(ck) if max_nc else None,
+        _ptr(cv) if max_nc else None, max_nc, _stream(k_new.device)))
+
+
+def decode_step(q: torch.Tensor, g: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                s_new: torch.Tensor, ctx_len: torch.Tensor, wk: torch.Tensor, wv: torch.Tensor,
+                ws: torch.Tensor, ck: torch.Tensor, cv: torch.Tensor,
+                scale: Optional[float] = None, workspace: Optional[torch.Tensor] = None,
+                out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One serving step: cache_append of the new tokens, then decode of their
+    queries q, g [S, 64, 512] against the updated cache."""
+    S, max_nc = _check_append(k_new, v_new, s_new, ctx_len, wk, wv, ws, ck, cv)
+    _check(q, "q", (S, HEADS, HEAD_DIM))
+    _check(g, "g", (S, HEADS, HEAD_DIM))
+    if scale is None:
+        scale = 1.0 / math.sqrt(HEAD_DIM)
+    if workspace is None:
+        workspace = decode_workspace(S, q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(out, "out", (S, HEADS, HEAD_DIM))
+    _check(workspace, "workspace", dtype=torch.uint8)
+    _ok("hca_decode_step", lib().hca_decode_step(
+        q.data_ptr(), g.data_ptr(), k_new.data_ptr(), v_new.data_ptr(), s_new.data_ptr(),
+        ctx_len.data_ptr(), S, HEADS, ctypes.c_float(scale), wk.data_ptr(), wv.data_ptr(),
+        ws.data_ptr(), _ptr(ck) if max_nc else None, _ptr(cv) if max_nc else None, max_nc,
+        workspace.data_ptr(), workspace.numel(), out.data_ptr(), _stream(q.device)))
     return out
 
 

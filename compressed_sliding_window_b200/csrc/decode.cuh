@@ -497,7 +497,10 @@ __device__ __forceinline__ void combine_cta(const Params& p, const long long* ti
           off += sz;
         }
       }
-      if (!mbar_wait_warp(bar_comb, nbatch & 1, abort_flag, kWaitLimitNs, 71)) return;
+      if (!mbar_wait_warp(bar_comb, nbatch & 1, abort_flag, kWaitLimitNs, 71)) {
+        if (lane == 0) abort_drain(abort_flag);   // this batch's copies may still land
+        return;
+      }
       ++nbatch;
       const int nAb = max(0, min(fe, A.n) - fs);  // runs of sequence A in this batch
       // Per row: the batch's largest m first (lane u reads split fs + u, then a
@@ -970,6 +973,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   }  // A0 < A1
+  if (threadIdx.x == 0) abort_drain(abort_flag);
   __syncthreads();
   if (warp == 2) {
     tc_fence_after();

@@ -17,6 +17,7 @@
 #include "compress.cuh"
 #include "prefill3.cuh"
 #include "decode.cuh"
+#include "append.cuh"
 
 namespace {
 
@@ -408,6 +409,46 @@ hca_status_t hca_decode_noalloc(const hca_bf16* q, const hca_bf16* ck, const hca
 
   if (launch_decode(maps, prm, grid, stream) != cudaSuccess) return HCA_ERR_CUDA;
   return launch_status();
+}
+
+hca_status_t hca_cache_append(const hca_bf16* k_new, const hca_bf16* v_new,
+                              const hca_bf16* s_new, const int32_t* ctx_len, int S, hca_bf16* wk,
+                              hca_bf16* wv, hca_bf16* ws, hca_bf16* ck, hca_bf16* cv, int max_nc,
+                              hca_stream_t stream) {
+  if (S < 1 || max_nc < 0) return HCA_ERR_INVALID_ARG;
+  if (k_new == nullptr || v_new == nullptr || s_new == nullptr || ctx_len == nullptr ||
+      wk == nullptr || wv == nullptr || ws == nullptr)
+    return HCA_ERR_INVALID_ARG;
+  if (max_nc > 0 && (ck == nullptr || cv == nullptr)) return HCA_ERR_INVALID_ARG;
+  const void* ptrs[6] = {k_new, v_new, wk, wv, ck, cv};
+  for (const void* ptr : ptrs)
+    if (ptr != nullptr && !aligned16(ptr)) return HCA_ERR_INVALID_ARG;
+  if (S > 0x7fffffff / HCA_WINDOW) return HCA_ERR_UNSUPPORTED;
+  hca::append::append_kernel<<<S, hca::append::kThreads, 0, stream>>>(
+      k_new, v_new, s_new, ctx_len, wk, wv, ws, ck, cv, max_nc);
+  return launch_status();
+}
+
+hca_status_t hca_decode_step(const hca_bf16* q, const hca_bf16* g, const hca_bf16* k_new,
+                             const hca_bf16* v_new, const hca_bf16* s_new,
+                             const int32_t* ctx_len, int S, int H, float scale, hca_bf16* wk,
+                             hca_bf16* wv, hca_bf16* ws, hca_bf16* ck, hca_bf16* cv, int max_nc,
+                             void* workspace, size_t ws_bytes, hca_bf16* out,
+                             hca_stream_t stream) {
+  // validate both halves before launching either
+  if (H != HCA_NUM_HEADS) return HCA_ERR_UNSUPPORTED;
+  if (S < 1 || max_nc < 0 || !scale_ok(scale)) return HCA_ERR_INVALID_ARG;
+  if (S > 65535) return HCA_ERR_UNSUPPORTED;
+  if (q == nullptr || g == nullptr || out == nullptr || workspace == nullptr)
+    return HCA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(g) || !aligned16(out)) return HCA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return HCA_ERR_INVALID_ARG;
+  if (ws_bytes < hca_decode_workspace_size(S)) return HCA_ERR_INVALID_ARG;
+  hca_status_t st =
+      hca_cache_append(k_new, v_new, s_new, ctx_len, S, wk, wv, ws, ck, cv, max_nc, stream);
+  if (st != HCA_OK) return st;
+  return hca_decode(q, ck, cv, max_nc, wk, wv, ctx_len, g, S, H, scale, workspace, ws_bytes, out,
+                    stream);
 }
 
 hca_status_t hca_get_device_error(hca_stream_t stream, unsigned int* where) {

@@ -102,6 +102,18 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   return mbar_wait_slow(bar, parity, abort_flag, limit_ns, where);
 }
 
+// After a bounded wait gave up (the abort flag is set), copies this CTA issued
+// earlier may still be writing its shared memory, and a CTA must not exit
+// (or reuse that memory) under them: wait 200 us, far longer than any copy
+// takes to land, before the CTA's final barrier.  No cost on a normal run.
+__device__ __forceinline__ void abort_drain(volatile int* abort_flag) {
+  if (*abort_flag) {
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 200000ull) {
+    }
+  }
+}
+
 // Warp-collective bounded wait: every lane of the warp gets the same answer,
 // so warp-synchronous code after it stays convergent even if the limit runs
 // out for some lanes while the phase completes for others.

@@ -821,14 +821,7 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
   }
 
   __syncwarp();
-  // On an aborted run (a bounded wait gave up), copies already issued may
-  // still be writing this CTA's shared memory: give them time to land before
-  // the CTA can exit.
-  if (threadIdx.x == 0 && *abort_flag) {
-    const uint64_t t0 = globaltimer_ns();
-    while (globaltimer_ns() - t0 < 200000ull) {
-    }
-  }
+  if (threadIdx.x == 0) abort_drain(abort_flag);
   cluster_sync_all();  // no CTA leaves while a peer may still touch its shared memory or TMEM
   if (warp == 2) {
     tc_fence_after();

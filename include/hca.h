@@ -173,6 +173,49 @@ hca_status_t hca_decode_noalloc(const hca_bf16* q, const hca_bf16* ck, const hca
                                 float scale, hca_bf16* out, hca_stream_t stream);
 
 /*
+ * hca_cache_append — incremental update of a decode cache by one new token per
+ * sequence (the step on either side of hca_decode in serving).
+ *   'BaiduがERNIE 5.5 Flash Baseを公開' §2.1: every 128 tokens become one
+ *   cache entry; the xenospectrum analysis (section 活性140億パラメータと
+ *   長文処理を支える仕組み): the newest 128 tokens stay raw.
+ *   For sequence i with L = ctx_len[i] (which counts the new token, at
+ *   position p = L - 1):
+ *     wk[i, p mod 128] = k_new[i];  wv[i, p mod 128] = v_new[i];
+ *     ws[i, p mod 128] = s_new[i]                       (the ring of raw tokens)
+ *   and when L is a multiple of 128, block j = L/128 - 1 (now exactly the ring)
+ *   is compressed into entry j:
+ *     w = softmax(ws[i, 0:128]) (fp32);  ck[i, j] = sum_r w_r wk[i, r];
+ *     cv[i, j] = sum_r w_r wv[i, r]           (fp32 accumulate, bf16 RNE)
+ *   -- the value hca_compress gives for that block of the raw sequence.
+ * Layout:  k_new, v_new [S, 512] bf16;  s_new [S] bf16;  ctx_len [S] int32 on
+ *          the device;  wk, wv [S, 128, 512] bf16 and ws [S, 128] bf16 rings,
+ *          updated in place;  ck, cv [S, max_nc, 512] bf16, entry j written in
+ *          place (may be NULL when max_nc = 0).
+ * Errors:  host-checked: S < 1, max_nc < 0, a null or (for the 512-wide
+ *          tensors) misaligned pointer -> HCA_ERR_INVALID_ARG.  A device-side
+ *          ctx_len < 1, or a completed block j >= max_nc, writes nothing for
+ *          that sequence (ctx_len < 1) or skips the entry, and is reported by
+ *          hca_get_device_error() as HCA_ERR_DEVICE_INPUT.
+ */
+hca_status_t hca_cache_append(const hca_bf16* k_new, const hca_bf16* v_new,
+                              const hca_bf16* s_new, const int32_t* ctx_len, int S, hca_bf16* wk,
+                              hca_bf16* wv, hca_bf16* ws, hca_bf16* ck, hca_bf16* cv, int max_nc,
+                              hca_stream_t stream);
+
+/*
+ * hca_decode_step — one serving step: hca_cache_append of the new tokens,
+ * then hca_decode of their queries against the updated cache, in stream
+ * order on `stream` (two launches).  Arguments as in those two calls;
+ * everything is validated before either kernel is launched.
+ */
+hca_status_t hca_decode_step(const hca_bf16* q, const hca_bf16* g, const hca_bf16* k_new,
+                             const hca_bf16* v_new, const hca_bf16* s_new,
+                             const int32_t* ctx_len, int S, int H, float scale, hca_bf16* wk,
+                             hca_bf16* wv, hca_bf16* ws, hca_bf16* ck, hca_bf16* cv, int max_nc,
+                             void* workspace, size_t ws_bytes, hca_bf16* out,
+                             hca_stream_t stream);
+
+/*
  * hca_get_device_error — synchronises `stream`, then reads and clears the
  * device-side error word of the current device.  Returns HCA_OK,
  * HCA_ERR_TIMEOUT, HCA_ERR_DEVICE_INPUT or HCA_ERR_CUDA.  `where`, if not

@@ -1,7 +1,7 @@
 """CPU fp64 oracle for HCA.  Test infrastructure only: the product path never
 imports this package (see ``oracle.hca_oracle``)."""
 from .hca_oracle import (  # noqa: F401
-    BLOCK, HEADS, HEAD_DIM, WINDOW, attend, block_weights, compress,
+    BLOCK, HEADS, HEAD_DIM, WINDOW, attend, block_weights, cache_append, compress,
     decode_forward, decode_keys, num_visible_blocks, prefill_forward,
     round_bf16, sigmoid, visited_pairs, window_start,
 )

@@ -252,6 +252,35 @@ def decode_forward(q, ck, cv, wk, wv, ctx_len, g, blk: int = BLOCK,
 
 
 # ---------------------------------------------------------------------------
+# Incremental cache update (serving)
+# ---------------------------------------------------------------------------
+def cache_append(wk, wv, ws, ck, cv, k_new, v_new, s_new, L: int,
+                 blk: int = BLOCK, win: int = WINDOW) -> None:
+    """One serving step of one sequence's decode cache, in place (fp64 arrays).
+
+    wk, wv: [win, D] and ws: [win] hold the raw window as a ring (token at
+    position p in slot p mod win); ck, cv: [max_nc, D] the compressed entries.
+    The new token sits at position p = L - 1: it is written to slot p mod win.
+    When L is a multiple of blk, block j = L // blk - 1 has just completed, and
+    with win == blk the ring then holds exactly that block, so entry j is the
+    block's softmax(s)-weighted sum taken from the ring ('BaiduがERNIE 5.5
+    Flash Baseを公開' §2.1: one cache entry per 128 tokens; xenospectrum
+    analysis: the newest 128 tokens stay raw).
+    """
+    if win != blk:
+        raise ValueError("the ring holds one whole block only when win == blk")
+    slot = (L - 1) % win
+    wk[slot] = k_new
+    wv[slot] = v_new
+    ws[slot] = s_new
+    if L % blk == 0:
+        j = L // blk - 1
+        w = block_weights(np.asarray(ws, dtype=np.float64))
+        ck[j] = w @ np.asarray(wk, dtype=np.float64)
+        cv[j] = w @ np.asarray(wv, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
 # Work counts (used for FLOP accounting and by the tests)
 # ---------------------------------------------------------------------------
 def visited_pairs(T: int, blk: int = BLOCK, win: int = WINDOW) -> int:

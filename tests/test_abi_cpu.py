@@ -34,7 +34,8 @@ def test_every_declared_symbol_is_exported(lib):
 def test_expected_entry_points_declared():
     names = set(declared_functions())
     for n in ("hca_compress", "hca_prefill_fwd", "hca_decode", "hca_decode_workspace_size",
-              "hca_get_device_error", "hca_status_string", "hca_version"):
+              "hca_get_device_error", "hca_status_string", "hca_version", "hca_cache_append",
+              "hca_decode_step"):
         assert n in names
 
 
@@ -98,6 +99,41 @@ def test_decode_rejects_bad_args(lib):
     assert lib.hca_decode(f, f, f, -1, f, f, f, f, 4, 64, 0.04, f, 1 << 30, f, None) == 1
     assert lib.hca_decode(f, f, f, 8, f, f, f, f, 4, 64, 0.0, f, 1 << 30, f, None) == 1
     assert lib.hca_decode(f, f, f, 8, f, f, f, f, 4, 64, 0.04, f + 16, 1 << 30, f, None) == 1
+
+
+def test_cache_append_and_decode_step_reject_bad_arguments(lib):
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    lib.hca_cache_append.argtypes = [vp, vp, vp, vp, i, vp, vp, vp, vp, vp, i, vp]
+    f = 1 << 20   # aligned fake device address; every call below is rejected on the host
+    ok_args = [f, f, f, f, 4, f, f, f, f, f, 8, None]
+
+    def append(**kw):
+        a = list(ok_args)
+        for idx, val in kw.items():
+            a[int(idx[1:])] = val
+        return lib.hca_cache_append(*a)
+    assert append(a4=0) == 1                 # S < 1
+    assert append(a10=-1) == 1               # max_nc < 0
+    assert append(a0=None) == 1              # no k_new
+    assert append(a3=None) == 1              # no ctx_len
+    assert append(a7=None) == 1              # no score ring
+    assert append(a8=None) == 1              # entries needed (max_nc > 0) but no ck
+    assert append(a5=f + 8) == 1             # misaligned ring
+    lib.hca_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i, i, ctypes.c_float, vp, vp, vp, vp,
+                                    vp, i, vp, ctypes.c_size_t, vp, vp]
+    base = [f, f, f, f, f, f, 4, 64, 0.04, f, f, f, f, f, 8, f, 1 << 30, f, None]
+
+    def step(**kw):
+        a = list(base)
+        for idx, val in kw.items():
+            a[int(idx[1:])] = val
+        return lib.hca_decode_step(*a)
+    assert step(a7=32) == 2                  # H != 64
+    assert step(a8=0.0) == 1                 # scale
+    assert step(a0=None) == 1                # no q
+    assert step(a15=f + 16) == 1             # workspace not 256-byte aligned
+    assert step(a2=None) == 1                # no k_new (append half)
+    assert step(a6=70000) == 2               # S beyond what decode supports
 
 
 def test_selftest_rejects_bad_limit(lib):
