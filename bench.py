@@ -607,6 +607,43 @@ def bench_decode(cfg, dev, peaks, args):
     cache_bytes = keys * 2 * 512 * 2
     total_bytes = cache_bytes + 3 * S * 64 * 512 * 2
     gbs = cache_bytes / (ms / 1e3) / 1e9
+    # the same workload with its cache stored in FP8 (e4m3 codes + one fp32
+    # scale per row), quantized once on the GPU outside the timed region
+    qc = {n: hca.quantize_e4m3(t) for n, t in (("ck", ck), ("cv", cv), ("wk", wk), ("wv", wv))}
+    torch.cuda.synchronize()
+
+    def dec8():
+        hca.decode_e4m3(q, qc["ck"][0], qc["ck"][1], qc["cv"][0], qc["cv"][1], qc["wk"][0],
+                        qc["wk"][1], qc["wv"][0], qc["wv"][1], ctx, g, workspace=ws, out=out)
+    for _ in range(3):
+        dec8()
+    torch.cuda.synchronize()
+    times8 = []
+    for _ in range(args.decode_steps):
+        flush_l2(flush, clean)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        dec8()
+        b.record(stream)
+        b.synchronize()
+        times8.append(a.elapsed_time(b))
+    code, where = hca.device_error(dev)
+    if code != 0:
+        raise RuntimeError(f"device error {code} at {where} (fp8 decode)")
+    srt8 = sorted(times8)
+    ms8 = statistics.fmean(srt8[cut:len(srt8) - cut])
+    cache8 = keys * 2 * (512 + 4)
+    total8 = cache8 + 3 * S * 64 * 512 * 2
+    fp8 = {"ms_per_step": ms8, "tok_per_s": S / (ms8 / 1e3), "cache_bytes": cache8,
+           "cache_gbs": cache8 / (ms8 / 1e3) / 1e9,
+           "roofline": {"bound": "hbm", "achieved": total8 / (ms8 / 1e3) / 1e9,
+                        "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": total8 / (ms8 / 1e3) / 1e9 / peaks["hbm_gbs"],
+                        "peak_source": peaks["source"]},
+           "storage": "e4m3 codes + one fp32 scale per 512-wide row (hca_quantize_e4m3)",
+           "speedup_vs_bf16_cache": ms / ms8}
+    del qc
     res = {"workload": cfg.name, "S": S, "ctx_len": lens if len(set(lens)) > 1 else lens[0],
            "tok_per_s": S / (ms / 1e3), "ms_per_step": ms, "cache_gbs": gbs,
            "total_gbs": total_bytes / (ms / 1e3) / 1e9,
@@ -616,7 +653,7 @@ def bench_decode(cfg, dev, peaks, args):
                         "peak_source": peaks["source"]},
            "l2": "flushed before every timed step (256 MB write, then 256 MB read)",
            "timing": f"CUDA events per step; mean of the middle 80 % of {len(times)} steps",
-           "gpu_launches_per_step": 1 if S <= 1024 else 2}
+           "gpu_launches_per_step": 1 if S <= 1024 else 2, "fp8_cache": fp8}
     del ck, cv, wk, wv, flush, clean, ws
     torch.cuda.empty_cache()
     return res
@@ -645,8 +682,14 @@ def run_profile_case(args):
         ck, cv = rnd(S, nc, 512), rnd(S, nc, 512)
         wk, wv, q, gg = rnd(S, 128, 512), rnd(S, 128, 512), rnd(S, 64, 512), rnd(S, 64, 512)
         ctx = torch.tensor(lens, dtype=torch.int32, device=dev)
-        for _ in range(args.warmup):
-            hca.decode(q, ck, cv, wk, wv, ctx, gg)
+        if dims and dims[0] == "fp8":
+            c = [hca.quantize_e4m3(t) for t in (ck, cv, wk, wv)]
+            for _ in range(args.warmup):
+                hca.decode_e4m3(q, c[0][0], c[0][1], c[1][0], c[1][1], c[2][0], c[2][1], c[3][0],
+                                c[3][1], ctx, gg)
+        else:
+            for _ in range(args.warmup):
+                hca.decode(q, ck, cv, wk, wv, ctx, gg)
     elif kind == "decode":
         S, L = int(dims[0]), int(dims[1])
         nc = L // 128
@@ -727,7 +770,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=50)
     ap.add_argument("--side-steps", type=int, default=20)
     ap.add_argument("--profile-case", default=None,
-                    help="prefill:T, decode:S:L or decode-long -- a few untimed launches for ncu")
+                    help="prefill:T, decode:S:L, decode-long or decode-long:fp8 -- a few untimed "
+                         "launches for ncu")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     if args.profile_case:

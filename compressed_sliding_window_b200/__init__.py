@@ -57,13 +57,17 @@ def lib() -> ctypes.CDLL:
         L.hca_cache_append.argtypes = [vp, vp, vp, vp, i, vp, vp, vp, vp, vp, i, vp]
         L.hca_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i, i, f, vp, vp, vp, vp, vp, i, vp,
                                       sz, vp, vp]
+        L.hca_quantize_e4m3.argtypes = [vp, ctypes.c_longlong, vp, vp, vp]
+        L.hca_decode_e4m3.argtypes = [vp, vp, vp, vp, vp, i, vp, vp, vp, vp, vp, vp, i, i, f, vp,
+                                      sz, vp, vp]
         L.hca_get_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
         L.hca_selftest_bounded_wait.argtypes = [i, vp]
         L.hca_status_string.argtypes = [i]
         L.hca_status_string.restype = ctypes.c_char_p
         L.hca_version.restype = i
         for name in ("hca_compress", "hca_prefill_fwd", "hca_decode", "hca_get_device_error",
-                     "hca_selftest_bounded_wait", "hca_cache_append", "hca_decode_step"):
+                     "hca_selftest_bounded_wait", "hca_cache_append", "hca_decode_step",
+                     "hca_quantize_e4m3", "hca_decode_e4m3"):
             getattr(L, name).restype = i
         _LIB = L
     return _LIB
@@ -258,6 +262,57 @@ def decode_step(q: torch.Tensor, g: torch.Tensor, k_new: torch.Tensor, v_new: to
         ctx_len.data_ptr(), S, HEADS, ctypes.c_float(scale), wk.data_ptr(), wv.data_ptr(),
         ws.data_ptr(), _ptr(ck) if max_nc else None, _ptr(cv) if max_nc else None, max_nc,
         workspace.data_ptr(), workspace.numel(), out.data_ptr(), _stream(q.device)))
+    return out
+
+
+def quantize_e4m3(x: torch.Tensor) -> Tuple[torch.Tensor, torch.Tensor]:
+    """FP8 storage of bf16 rows x [..., 512]: (codes uint8 [..., 512], scale
+    fp32 [...]), scale = amax / 448 per row, codes = e4m3(x / scale)."""
+    if x.shape[-1] != HEAD_DIM:
+        raise ValueError(f"x rows must be {HEAD_DIM} wide")
+    _check(x, "x", tuple(x.shape))
+    codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    scale = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    rows = x.numel() // HEAD_DIM
+    _ok("hca_quantize_e4m3", lib().hca_quantize_e4m3(
+        x.data_ptr(), rows, codes.data_ptr(), scale.data_ptr(), _stream(x.device)))
+    return codes, scale
+
+
+def decode_e4m3(q: torch.Tensor, ck: torch.Tensor, ck_scale: torch.Tensor, cv: torch.Tensor,
+                cv_scale: torch.Tensor, wk: torch.Tensor, wk_scale: torch.Tensor,
+                wv: torch.Tensor, wv_scale: torch.Tensor, ctx_len: torch.Tensor, g: torch.Tensor,
+                scale: Optional[float] = None, workspace: Optional[torch.Tensor] = None,
+                out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One decode step over an FP8 cache (codes and row scales from
+    ``quantize_e4m3``): q, g [S, 64, 512] bf16; ck, cv [S, max_nc, 512] codes
+    with [S, max_nc] scales; wk, wv [S, 128, 512] ring codes with [S, 128]
+    scales; ctx_len [S] int32."""
+    S, H, D = q.shape
+    _check(q, "q", (S, H, HEAD_DIM))
+    _check(g, "g", (S, H, HEAD_DIM))
+    max_nc = ck.shape[1]
+    for t, n, shp in ((ck, "ck", (S, max_nc, HEAD_DIM)), (cv, "cv", (S, max_nc, HEAD_DIM)),
+                      (wk, "wk", (S, WINDOW, HEAD_DIM)), (wv, "wv", (S, WINDOW, HEAD_DIM))):
+        _check(t, n, shp, dtype=torch.uint8)
+    for t, n, shp in ((ck_scale, "ck_scale", (S, max_nc)), (cv_scale, "cv_scale", (S, max_nc)),
+                      (wk_scale, "wk_scale", (S, WINDOW)), (wv_scale, "wv_scale", (S, WINDOW))):
+        _check(t, n, shp, dtype=torch.float32)
+    _check(ctx_len, "ctx_len", (S,), dtype=torch.int32)
+    if scale is None:
+        scale = 1.0 / math.sqrt(HEAD_DIM)
+    if workspace is None:
+        workspace = decode_workspace(S, q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(out, "out", (S, H, HEAD_DIM))
+    _check(workspace, "workspace", dtype=torch.uint8)
+    _ok("hca_decode_e4m3", lib().hca_decode_e4m3(
+        q.data_ptr(), _ptr(ck) if max_nc else None, _ptr(ck_scale) if max_nc else None,
+        _ptr(cv) if max_nc else None, _ptr(cv_scale) if max_nc else None, max_nc,
+        wk.data_ptr(), wk_scale.data_ptr(), wv.data_ptr(), wv_scale.data_ptr(),
+        ctx_len.data_ptr(), g.data_ptr(), S, H, ctypes.c_float(scale), workspace.data_ptr(),
+        workspace.numel(), out.data_ptr(), _stream(q.device)))
     return out
 
 

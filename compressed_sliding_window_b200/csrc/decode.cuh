@@ -24,8 +24,21 @@
 // M = 64; instead keys go on the 128-lane M axis:
 //   S^T[key, head] = K_tile[key, :] . Q[head, :]        (M=128, N=64, K=512)
 //   O^T[dv, head] += V_tile[:, dv]^T . P^T[:, head]      (4 x M=128 dv, N=64, K=128)
-// TMEM holds O^T (4 x 64 columns) and two 64-column S^T buffers.  The softmax
-// runs across lanes: each thread owns one key and its 64 head scores, and the
+// TMEM holds O^T (4 x 64 columns) and two 64-column S^T buffers.
+//
+// FP8 cache (decode_kernel<true>).  The cache rows are e4m3 codes with one
+// fp32 scale per row (half the bytes to stream).  Each producer warp loads
+// 16 KB code tiles (128 keys x 128 channels) into its own staging slots and,
+// with all 32 lanes, turns a landed tile into its f16 ring stage (a few
+// integer operations and one f16x2 multiply per two values: every e4m3 value
+// is exact in f16); Q is turned from bf16 into f16 in place by the softmax
+// warps at each segment start (exact for |q| < 65504), and the MMAs run in
+// f16.  Each softmax thread owns one key: it multiplies its scores by the
+// key's K scale and its probabilities by the key's V scale before they feed
+// P.V (the row sums use the unscaled probabilities), so no scaling touches
+// the operand tiles.
+//
+// The softmax runs across lanes: each thread owns one key and its 64 head scores, and the
 // per-head max / sum over the 128 keys come from a shuffle transpose-reduce
 // (62 shuffles per warp) plus one small shared-memory step.
 #pragma once
@@ -44,7 +57,10 @@ constexpr int kSlab = 16384;        // [128 keys x 64 bf16] swizzled
 constexpr int kStage = 2 * kSlab;   // one copy: two 64-wide slabs of a 128-key tile
 constexpr int kQSlab = 8192;        // [64 heads x 64 bf16] swizzled
 constexpr int kSmemQ = 0;           // 8 x 8 KB
-constexpr int kSmemRing = 65536;    // 4 x 32 KB
+constexpr int kSmemRing = 65536;    // 4 x 32 KB (FP8 cache: 2 x 32 KB, then 4 x 16 KB staging)
+constexpr int kStagesF8 = 2;
+constexpr int kStgBytes = 16384;    // one FP8 code tile: [128 keys][128 bytes]
+constexpr int kSmemStg = kSmemRing + kStagesF8 * 2 * kSlab;
 constexpr int kSmemPT = kSmemRing + kStages * kStage;  // P^T [128 keys x 64 heads] bf16, 16 KB
 constexpr int kSmemRed = kSmemPT + 16384;             // reductions, 4 KB
 constexpr int kSmemBar = kSmemRed + 4096;
@@ -70,11 +86,13 @@ constexpr int R_FLAG = 768;         // ints: [0] ok, [1] any-rescale
 enum {
   B_QFULL = 0, B_QEMPTY = 1, B_FULL = 2, B_EMPTY = B_FULL + kStages, B_SFULL = B_EMPTY + kStages,
   B_SFREE = B_SFULL + 2, B_PFULL = B_SFREE + 2, B_PFREE = B_PFULL + 1, B_OFULL = B_PFREE + 1,
-  B_OFREE = B_OFULL + 1, B_DRAIN = B_OFREE + 1, B_COMB = B_DRAIN + 1, B_COUNT = B_COMB + 1
+  B_OFREE = B_OFULL + 1, B_DRAIN = B_OFREE + 1, B_COMB = B_DRAIN + 1, B_STG = B_COMB + 1,
+  B_QCONV = B_STG + 4, B_COUNT = B_QCONV + 1
 };
 constexpr int kTmemSlot = 8 * B_COUNT;
 constexpr int kAbortSlot = kTmemSlot + 4;
 static_assert(kAbortSlot + 4 <= 256, "barrier region overflow");
+static_assert(kSmemStg + 4 * kStgBytes == kSmemRing + kStages * 2 * 16384, "FP8 layout");
 
 constexpr uint32_t kTmemO = 0, kTmemS0 = 256, kTmemS1 = 320, kTmemCols = 512;
 
@@ -100,6 +118,11 @@ struct Params {
   unsigned long long* gsync;  // grid barrier arrivals (zero before first use, see below)
   const uint16_t* g;   // [S, 64, 512] bf16 gate
   uint16_t* out;       // [S, 64, 512] bf16
+  // FP8 cache only: per-row scales of ck, cv [S, max_nc] and wk, wv [S, 128]
+  const float* sck;
+  const float* scv;
+  const float* swk;
+  const float* swv;
 };
 
 __device__ __forceinline__ int nc_of_len(int L) { return L >= 128 ? (L - 128) / 128 : 0; }
@@ -237,6 +260,8 @@ __device__ __forceinline__ void inline_plan(const Params& p, long long* sT, int*
 
 // 4-D views (64, rows, 8 slabs, S) of [S][rows][512] tensors: a box
 // (64, rows, n, 1) lands as n 64-wide slabs of [rows][64], 128B-swizzled.
+// (FP8 cache: ck, cv, wk, wv are [S][rows][512 bytes] code maps, box
+// (128 bytes, 128 rows, 1), no swizzle.)
 struct Maps {
   CUtensorMap q;    // (64, S*64, 8, 1),  box (64, 64, 8, 1): the whole q of one sequence
   CUtensorMap ck;   // (64, max_nc, 8, S), box (64, 128, 2, 1)
@@ -586,8 +611,33 @@ __device__ __forceinline__ void combine_cta(const Params& p, const long long* ti
   }
 }
 
+// Four e4m3 codes (one word, lowest address in the low byte) -> four f16
+// values, exactly, with integer operations.  Each code moves into its own
+// 16-bit lane shifted left by 7: its exponent and mantissa bits then sit where
+// f16 keeps them (the f16 value is 2^-8 times the code's value; e4m3
+// subnormals land on f16 subnormals); its sign bit, now at bit 14, moves to
+// bit 15 by adding bit 14 to itself (no carry leaves the lane); one f16x2
+// multiply by 2^8 restores the value.
+__device__ __forceinline__ uint32_t mul_f16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const uint32_t a = __byte_perm(w, 0u, 0x4140) << 7;   // codes 0, 1
+  const uint32_t b = __byte_perm(w, 0u, 0x4342) << 7;   // codes 2, 3
+  lo = mul_f16x2(a + (a & 0x40004000u), 0x5C005C00u);   // x 256 (f16 0x5C00)
+  hi = mul_f16x2(b + (b & 0x40004000u), 0x5C005C00u);
+}
+// a bf16 pair -> an f16 pair (exact for |x| < 65504 with at most 11 significant bits)
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+  return pack_f16x2(bf16lo_to_f32(w), bf16hi_to_f32(w));
+}
+
+template <bool kF8>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ Maps maps, const Params p) {
+  constexpr int NS = kF8 ? kStagesF8 : kStages;   // ring stages
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned, derived from smem_raw itself so that the compiler
   // keeps accesses through it in the shared state space
@@ -608,9 +658,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar(B_QFULL), 1);
     mbar_init(bar(B_QEMPTY), 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(bar(B_FULL + s), 1);
       mbar_init(bar(B_EMPTY + s), 1);
+    }
+    if (kF8) {
+      for (int s = 0; s < 4; ++s) mbar_init(bar(B_STG + s), 1);
+      mbar_init(bar(B_QCONV), 4);   // one arrive per softmax warp
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(B_SFULL + s), 1);
@@ -660,7 +714,117 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Segments: maximal runs of this CTA's tiles inside one sequence.
   const int s_first = find_seq(tiles, p.S, A0);
 
-  if (warp <= 1) {
+  if (warp <= 1 && kF8) {
+    // ------------------------------------------------------------ producers, FP8 cache
+    // Each warp loads the code tiles of its ring uses (alternate uses, as
+    // below) into its two staging slots, keeping up to two in flight, and
+    // converts each landed tile into its ring stage with all 32 lanes.
+    const int me = warp;
+    const uint32_t sStg = sbase + kSmemStg;
+    uint32_t u = 0, quse = 0, nown = 0, first = 0, npend = 0;
+    bool ok = true;
+    // convert this warp's oldest pending use (own use index `first`)
+    auto convert_oldest = [&]() -> bool {
+      const uint32_t slot = first & 1;
+      const uint32_t uu = 2 * first + static_cast<uint32_t>(me);
+      const uint32_t st = uu % NS;
+      bool w_ok = true;
+      if (lane == 0)
+        w_ok = mbar_wait(bar(B_STG + 2 * me + slot), (first >> 1) & 1, abort_flag, kWaitLimitNs,
+                         42) &&
+               mbar_wait(bar(B_EMPTY + st), ((uu / NS) & 1) ^ 1, abort_flag, kWaitLimitNs, 40);
+      w_ok = __shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0) != 0;
+      if (!w_ok) return false;
+      mbar_try_wait(bar(B_STG + 2 * me + slot), (first >> 1) & 1);   // this lane's acquire
+      const uint8_t* src = smem + kSmemStg + (2 * me + slot) * kStgBytes;
+      uint8_t* dst = smem + kSmemRing + st * kStage;
+      // 16-byte source chunk ci (16 codes): key row ci / 8, bytes 16 (ci % 8) of
+      // the 128-channel row, i.e. slab (ci % 8) / 4 and 16-byte output chunks
+      // 2 (ci % 4) and 2 (ci % 4) + 1 of that slab's row
+#pragma unroll 2
+      for (int it = 0; it < 32; ++it) {
+        const int ci = it * 32 + lane;
+        const int row = ci >> 3, sl = (ci >> 2) & 1, c = (ci & 3) * 2;
+        const uint4 x = *reinterpret_cast<const uint4*>(src + ci * 16);
+        uint32_t f[8];
+        e4m3x4_to_f16x4(x.x, f[0], f[1]);
+        e4m3x4_to_f16x4(x.y, f[2], f[3]);
+        e4m3x4_to_f16x4(x.z, f[4], f[5]);
+        e4m3x4_to_f16x4(x.w, f[6], f[7]);
+        uint8_t* drow = dst + sl * kSlab;
+        *reinterpret_cast<uint4*>(drow + sw128_offset(row, c)) = make_uint4(f[0], f[1], f[2], f[3]);
+        *reinterpret_cast<uint4*>(drow + sw128_offset(row, c + 1)) =
+            make_uint4(f[4], f[5], f[6], f[7]);
+      }
+      fence_proxy_async_smem();   // read next by the tensor core (async proxy)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_FULL + st));
+      ++first;
+      --npend;
+      return true;
+    };
+    // code tile (channels [64 z, 64 z + 128), rows y..y+127) of use u
+    auto load = [&](const CUtensorMap* map, int y, int z, int w) -> bool {
+      if ((u & 1) == static_cast<uint32_t>(me)) {
+        if (npend == 2 && !convert_oldest()) return false;
+        const uint32_t slot = nown & 1;
+        if (lane == 0) {
+          mbar_expect_tx(bar(B_STG + 2 * me + slot), kStgBytes);
+          tma_load_3d(sStg + (2 * me + slot) * kStgBytes, map, bar(B_STG + 2 * me + slot), 64 * z,
+                      y, w);
+        }
+        ++nown;
+        ++npend;
+      }
+      ++u;
+      return true;
+    };
+    long long x = A0;
+    for (int s = s_first; x < A1 && ok; ++s) {
+      const SeqInfo si = seq_info(lens, p.max_nc, s);
+      const long long seg_end = min(A1, tiles[s + 1]);
+      const int j0 = static_cast<int>(x - tiles[s]);
+      const int j1 = static_cast<int>(seg_end - tiles[s]);
+      if (me == 0) {
+        if (lane == 0) {
+          ok = mbar_wait(bar(B_QEMPTY), (quse & 1) ^ 1, abort_flag, kWaitLimitNs, 41);
+          if (ok) {
+            mbar_expect_tx(bar(B_QFULL), 8 * kQSlab);
+            tma_load_4d_dec(sQ, &maps.q, bar(B_QFULL), 0, s * kHeads, 0, 0);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+      }
+      ++quse;
+      auto load_k = [&](int j) -> bool {
+        for (int d = 0; d < 4 && ok; ++d)
+          ok = (j < si.nct) ? load(&maps.ck, j * kKeyTile, 2 * d, s) : load(&maps.wk, 0, 2 * d, s);
+        return ok;
+      };
+      auto load_v = [&](int j) -> bool {
+        for (int e = 0; e < 4 && ok; ++e)
+          ok = (j < si.nct) ? load(&maps.cv, j * kKeyTile, 2 * e, s) : load(&maps.wv, 0, 2 * e, s);
+        return ok;
+      };
+      if (!load_k(j0)) break;
+      for (int j = j0; j < j1 && ok; ++j) {
+        if (j + 1 < j1 && !load_k(j + 1)) break;
+        if (!load_v(j)) break;
+      }
+      x = seg_end;
+    }
+    while (ok && npend > 0) ok = convert_oldest();
+    if (me == 0 && lane == 0) {
+      const long long R = static_cast<long long>(p.S) * kHeads;
+      const long long r0 = div_nn(R * blockIdx.x, gridDim.x);
+      const long long r1 = div_nn(R * (blockIdx.x + 1), gridDim.x);
+      if (r1 > r0)
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.g + r0 * kDim),
+                     "r"(static_cast<uint32_t>(r1 - r0) * kDim * 2)
+                     : "memory");
+    }
+  } else if (warp <= 1) {
     // ------------------------------------------------------------ producers
     // Two warps alternate ring stages: one issuing thread cannot keep enough
     // copies in flight to cover HBM latency.
@@ -670,8 +834,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       auto load = [&](const CUtensorMap* map, int y, int z, int w) -> bool {
         if ((u & 1) == static_cast<uint32_t>(me)) {
-          const uint32_t st = u % kStages;
-          if (!mbar_wait(bar(B_EMPTY + st), ((u / kStages) & 1) ^ 1, abort_flag, kWaitLimitNs, 40))
+          const uint32_t st = u % NS;
+          if (!mbar_wait(bar(B_EMPTY + st), ((u / NS) & 1) ^ 1, abort_flag, kWaitLimitNs, 40))
             return false;
           mbar_expect_tx(bar(B_FULL + st), kStage);
           tma_load_4d_dec(sRing + st * kStage, map, bar(B_FULL + st), 0, y, z, w);
@@ -726,8 +890,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t ring = 0, quse = 0, sidx = 0, pvidx = 0, nseg = 0;
       bool ok = true;
-      const uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
-      const uint32_t idesc_o = idesc_bf16_f32(128, 64, true, true);
+      const uint32_t idesc_s = kF8 ? idesc_f16_f32(128, 64, false, false)
+                                   : idesc_bf16_f32(128, 64, false, false);
+      const uint32_t idesc_o = kF8 ? idesc_f16_f32(128, 64, true, true)
+                                   : idesc_bf16_f32(128, 64, true, true);
       auto issue_s = [&]() -> bool {
         const uint32_t buf = sidx & 1;
         if (!mbar_wait(bar(B_SFREE + buf), ((sidx >> 1) & 1) ^ 1, abort_flag, kWaitLimitNs, 50))
@@ -735,8 +901,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t dS = tmem + (buf ? kTmemS1 : kTmemS0);
         for (int d2 = 0; d2 < 4; ++d2) {
-          const uint32_t st = ring % kStages;
-          if (!mbar_wait(bar(B_FULL + st), (ring / kStages) & 1, abort_flag, kWaitLimitNs, 51))
+          const uint32_t st = ring % NS;
+          if (!mbar_wait(bar(B_FULL + st), (ring / NS) & 1, abort_flag, kWaitLimitNs, 51))
             return false;
           tc_fence_after();
 #pragma unroll
@@ -762,8 +928,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           return false;
         tc_fence_after();
         for (int c = 0; c < 4; ++c) {
-          const uint32_t st = ring % kStages;
-          if (!mbar_wait(bar(B_FULL + st), (ring / kStages) & 1, abort_flag, kWaitLimitNs, 54))
+          const uint32_t st = ring % NS;
+          if (!mbar_wait(bar(B_FULL + st), (ring / NS) & 1, abort_flag, kWaitLimitNs, 54))
             return false;
           tc_fence_after();
 #pragma unroll
@@ -783,7 +949,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = s_first; x < A1 && ok; ++s) {
         const long long seg_end = min(A1, tiles[s + 1]);
         const int ntl = static_cast<int>(seg_end - x);
-        ok = mbar_wait(bar(B_QFULL), quse & 1, abort_flag, kWaitLimitNs, 56);
+        // FP8 cache: Q once the softmax warps turned it into f16
+        ok = mbar_wait(bar(kF8 ? B_QCONV : B_QFULL), quse & 1, abort_flag, kWaitLimitNs, 56);
         if (!ok) break;
         ++quse;
         tc_fence_after();
@@ -831,8 +998,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         red[R_MRUN + tid] = -INFINITY;
         red[R_LRUN + tid] = 0.f;
       }
+      if constexpr (kF8) {
+        // this segment's Q, bf16 -> f16 in place (same byte positions), for the MMA
+        if (!group_wait(bar(B_QFULL), nseg & 1, 63)) { ok = false; break; }
+        uint4* qa = reinterpret_cast<uint4*>(smem + kSmemQ);
+#pragma unroll 4
+        for (int i = 0; i < 8 * kQSlab / 16 / 128; ++i) {
+          uint4 w = qa[i * 128 + tid];
+          w = make_uint4(bf16x2_to_f16x2(w.x), bf16x2_to_f16x2(w.y), bf16x2_to_f16x2(w.z),
+                         bf16x2_to_f16x2(w.w));
+          qa[i * 128 + tid] = w;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_QCONV));
+      }
       for (int j = j0; j < j1; ++j) {
         const uint32_t buf = sidx & 1;
+        // FP8 cache: this key's row scales (loaded before the wait)
+        float sk = 1.f, sv = 1.f;
+        if constexpr (kF8) {
+          const bool comp = j < si.nct;
+          const int e = j * kKeyTile + key;
+          if (comp ? e < si.nc : ((si.L >= kWin) || (key < si.L))) {
+            const size_t ix = comp ? static_cast<size_t>(s) * p.max_nc + e
+                                   : static_cast<size_t>(s) * kWin + key;
+            sk = __ldg((comp ? p.sck : p.swk) + ix);
+            sv = __ldg((comp ? p.scv : p.swv) + ix);
+          }
+        }
         if (!group_wait(bar(B_SFULL + buf), (sidx >> 1) & 1, 60)) { ok = false; break; }
         tc_fence_after();
         uint32_t r[64];
@@ -850,8 +1044,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j < si.nct) valid = j * kKeyTile + key < si.nc;
         else valid = (si.L >= kWin) || (key < si.L);
         float a[64];
+        const float sc = p.scale_log2 * sk;
 #pragma unroll
-        for (int h = 0; h < 64; ++h) a[h] = valid ? __uint_as_float(r[h]) * p.scale_log2 : -INFINITY;
+        for (int h = 0; h < 64; ++h) a[h] = valid ? __uint_as_float(r[h]) * sc : -INFINITY;
         float xv[64];
 #pragma unroll
         for (int h = 0; h < 64; ++h) xv[h] = a[h];
@@ -888,7 +1083,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float e1 = ex2_approx(xv[h + 1] - red[R_MUSE + h + 1]);
           ps[h] = e0;
           ps[h + 1] = e1;
-          pk[h / 2] = pack_bf16x2(e0, e1);
+          // FP8 cache: the key's V scale rides on its probabilities (f16 P)
+          pk[h / 2] = kF8 ? pack_f16x2(e0 * sv, e1 * sv) : pack_bf16x2(e0, e1);
         }
         warp_transpose_reduce64<false>(ps);
         red[R_SUM + gw * 64 + 2 * lane] = ps[0];

@@ -18,6 +18,7 @@
 #include "prefill3.cuh"
 #include "decode.cuh"
 #include "append.cuh"
+#include "quant.cuh"
 
 namespace {
 
@@ -92,6 +93,20 @@ bool make_map_bytes(CUtensorMap* m, const void* base, uint64_t rows, uint32_t bo
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D byte view [Z][Y][512] of e4m3 code rows, box (128 bytes, 128 rows, 1),
+// no swizzle: one 128-channel, 128-key code tile.
+bool make_map_codes(CUtensorMap* m, const void* base, uint64_t Y, uint64_t Z) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[3] = {512, Y, Z};
+  const cuuint64_t strides[2] = {512, 512 * Y};
+  const cuuint32_t box[3] = {128, 128, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // How many 4-CTA clusters of the prefill kernel fit on the current device at
 // once.  The shared-memory attribute is a per-device property of the kernel,
 // so it is set, and the occupancy asked, once for every device the process
@@ -129,10 +144,11 @@ int prefill_max_clusters() {
 // (the decode kernel then starts early and waits for it inside), else the
 // decode kernel alone, which plans for itself.  Cooperative either way: the
 // kernel holds a grid barrier.
+template <bool kF8>
 cudaError_t launch_decode(const hca::decode::Maps& maps, const hca::decode::Params& prm, int grid,
                           cudaStream_t stream) {
   namespace D = hca::decode;
-  cudaError_t err = cudaFuncSetAttribute(D::decode_kernel,
+  cudaError_t err = cudaFuncSetAttribute(D::decode_kernel<kF8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, D::kSmemAlloc);
   if (err != cudaSuccess) return err;
   const bool inl = prm.S <= D::kInlineSeqs;
@@ -153,7 +169,7 @@ cudaError_t launch_decode(const hca::decode::Maps& maps, const hca::decode::Para
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = inl ? 1 : 2;
-  return cudaLaunchKernelEx(&cfg, D::decode_kernel, maps, prm);
+  return cudaLaunchKernelEx(&cfg, D::decode_kernel<kF8>, maps, prm);
 }
 
 hca_status_t launch_status() {
@@ -250,7 +266,7 @@ hca_status_t hca_prefill_fwd(const hca_bf16* q, const hca_bf16* k, const hca_bf1
   }
   if (!ok) return HCA_ERR_CUDA;
 
-  P::Params prm;
+  P::Params prm = {};
   prm.B = B;
   prm.T = T;
   prm.row_tiles = static_cast<int>(row_tiles);
@@ -295,7 +311,7 @@ hca_status_t hca_decode(const hca_bf16* q, const hca_bf16* ck, const hca_bf16* c
   if (sms <= 0) return HCA_ERR_CUDA;
   const int slots = sms + S;
   uint8_t* wsb = static_cast<uint8_t*>(ws);
-  D::Params prm;
+  D::Params prm = {};
   prm.ctx_len = ctx_len;
   prm.S = S;
   prm.max_nc = max_nc;
@@ -320,7 +336,7 @@ hca_status_t hca_decode(const hca_bf16* q, const hca_bf16* ck, const hca_bf16* c
   }
   if (!ok) return HCA_ERR_CUDA;
 
-  if (launch_decode(maps, prm, sms, stream) != cudaSuccess) return HCA_ERR_CUDA;
+  if (launch_decode<false>(maps, prm, sms, stream) != cudaSuccess) return HCA_ERR_CUDA;
   return launch_status();
 }
 
@@ -383,7 +399,7 @@ hca_status_t hca_decode_noalloc(const hca_bf16* q, const hca_bf16* ck, const hca
   uint8_t* wsb = static_cast<uint8_t*>(noalloc_scratch_address());
   if (wsb == nullptr) return HCA_ERR_CUDA;
 
-  D::Params prm;
+  D::Params prm = {};
   prm.ctx_len = ctx_len;
   prm.S = S;
   prm.max_nc = max_nc;
@@ -407,7 +423,7 @@ hca_status_t hca_decode_noalloc(const hca_bf16* q, const hca_bf16* ck, const hca
   }
   if (!ok) return HCA_ERR_CUDA;
 
-  if (launch_decode(maps, prm, grid, stream) != cudaSuccess) return HCA_ERR_CUDA;
+  if (launch_decode<false>(maps, prm, grid, stream) != cudaSuccess) return HCA_ERR_CUDA;
   return launch_status();
 }
 
@@ -449,6 +465,79 @@ hca_status_t hca_decode_step(const hca_bf16* q, const hca_bf16* g, const hca_bf1
   if (st != HCA_OK) return st;
   return hca_decode(q, ck, cv, max_nc, wk, wv, ctx_len, g, S, H, scale, workspace, ws_bytes, out,
                     stream);
+}
+
+hca_status_t hca_quantize_e4m3(const hca_bf16* x, long long rows, uint8_t* codes, float* scale,
+                               hca_stream_t stream) {
+  if (rows < 0 || (rows > 0 && (x == nullptr || codes == nullptr || scale == nullptr)))
+    return HCA_ERR_INVALID_ARG;
+  if (rows == 0) return HCA_OK;
+  if (!aligned16(x) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scale) & 3u) != 0)
+    return HCA_ERR_INVALID_ARG;
+  namespace Q = hca::quant;
+  const long long ctas = (rows + Q::kRowsPerCta - 1) / Q::kRowsPerCta;
+  if (ctas > 0x7fffffffLL) return HCA_ERR_UNSUPPORTED;
+  Q::quantize_e4m3_kernel<<<static_cast<unsigned>(ctas), Q::kThreads, 0, stream>>>(x, rows, codes,
+                                                                                   scale);
+  return launch_status();
+}
+
+hca_status_t hca_decode_e4m3(const hca_bf16* q, const uint8_t* ck, const float* ck_scale,
+                             const uint8_t* cv, const float* cv_scale, int max_nc,
+                             const uint8_t* wk, const float* wk_scale, const uint8_t* wv,
+                             const float* wv_scale, const int32_t* ctx_len, const hca_bf16* g,
+                             int S, int H, float scale, void* ws, size_t ws_bytes, hca_bf16* out,
+                             hca_stream_t stream) {
+  namespace D = hca::decode;
+  if (H != HCA_NUM_HEADS) return HCA_ERR_UNSUPPORTED;
+  if (S < 1 || max_nc < 0 || !scale_ok(scale)) return HCA_ERR_INVALID_ARG;
+  if (q == nullptr || wk == nullptr || wv == nullptr || wk_scale == nullptr ||
+      wv_scale == nullptr || ctx_len == nullptr || g == nullptr || out == nullptr || ws == nullptr)
+    return HCA_ERR_INVALID_ARG;
+  if (max_nc > 0 && (ck == nullptr || cv == nullptr || ck_scale == nullptr || cv_scale == nullptr))
+    return HCA_ERR_INVALID_ARG;
+  const void* ptrs[7] = {q, wk, wv, g, out, ck, cv};
+  for (const void* ptr : ptrs)
+    if (ptr != nullptr && !aligned16(ptr)) return HCA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return HCA_ERR_INVALID_ARG;
+  if (ws_bytes < hca_decode_workspace_size(S)) return HCA_ERR_INVALID_ARG;
+  if (static_cast<long long>(S) * HCA_NUM_HEADS > 0x7fffffffLL || S > 65535)
+    return HCA_ERR_UNSUPPORTED;
+
+  const int sms = device_sms();
+  if (sms <= 0) return HCA_ERR_CUDA;
+  const int slots = sms + S;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  D::Params prm = {};
+  prm.ctx_len = ctx_len;
+  prm.S = S;
+  prm.max_nc = max_nc;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.gsync = reinterpret_cast<unsigned long long*>(wsb);
+  prm.ws_o = reinterpret_cast<uint16_t*>(wsb + 256);
+  prm.ws_ml = reinterpret_cast<float*>(wsb + 256 + D::ws_o_bytes(slots));
+  prm.seq_tile =
+      reinterpret_cast<long long*>(wsb + 256 + ((D::ws_bytes(slots) + 255) & ~size_t(255)));
+  prm.g = g;
+  prm.out = out;
+  prm.sck = ck_scale;
+  prm.scv = cv_scale;
+  prm.swk = wk_scale;
+  prm.swv = wv_scale;
+
+  D::Maps maps;
+  bool ok = make_map4(&maps.q, q, static_cast<uint64_t>(S) * HCA_NUM_HEADS, 1, 64, 8) &&
+            make_map_codes(&maps.wk, wk, HCA_WINDOW, S) &&
+            make_map_codes(&maps.wv, wv, HCA_WINDOW, S);
+  if (ok && max_nc > 0) {
+    ok = make_map_codes(&maps.ck, ck, max_nc, S) && make_map_codes(&maps.cv, cv, max_nc, S);
+  } else if (ok) {
+    maps.ck = maps.wk;
+    maps.cv = maps.wv;
+  }
+  if (!ok) return HCA_ERR_CUDA;
+  if (launch_decode<true>(maps, prm, sms, stream) != cudaSuccess) return HCA_ERR_CUDA;
+  return launch_status();
 }
 
 hca_status_t hca_get_device_error(hca_stream_t stream, unsigned int* where) {

@@ -339,6 +339,12 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, bo
          ((b_mn ? 1u : 0u) << 16) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
+// The same for f16 A/B (format field 0).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(uint32_t M, uint32_t N, bool a_mn, bool b_mn) {
+  return (1u << 4) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) | ((N >> 3) << 17) |
+         ((M >> 4) << 24);
+}
+
 // ---------------------------------------------------------------------------
 // Thread-block clusters and distributed shared memory
 // ---------------------------------------------------------------------------
@@ -579,6 +585,31 @@ __device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int x, i
 // ---------------------------------------------------------------------------
 // Small numeric helpers
 // ---------------------------------------------------------------------------
+// Packed two-lane fp32 arithmetic (sm_100 f32x2): a * s + b and a + b.
+__device__ __forceinline__ float2 fma2(float2 a, float s, float b) {
+  float2 r;
+  asm("{.reg .b64 ap, sp, bp, rp;\n"
+      " mov.b64 ap, {%2, %3};\n"
+      " mov.b64 sp, {%4, %4};\n"
+      " mov.b64 bp, {%5, %5};\n"
+      " fma.rn.f32x2 rp, ap, sp, bp;\n"
+      " mov.b64 {%0, %1}, rp;}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(s), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 r;
+  asm("{.reg .b64 ap, bp, rp;\n"
+      " mov.b64 ap, {%2, %3};\n"
+      " mov.b64 bp, {%4, %5};\n"
+      " add.rn.f32x2 rp, ap, bp;\n"
+      " mov.b64 {%0, %1}, rp;}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+
 // 16-byte global load through the read-only path / plain 16-byte store
 __device__ __forceinline__ uint4 ld_nc_v4(const uint4* ptr) {
   uint4 v;

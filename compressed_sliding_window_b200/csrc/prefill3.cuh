@@ -414,9 +414,18 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
             tmem_ld32(sbase + cc, r);
             tmem_wait_ld_dep32(r);
             const int lo = clo - c0 - cc, hi = chi - c0 - cc;
+            if (lo <= 0 && hi >= 32) {   // warp-uniform: the whole chunk visible
+              float mx[4];
 #pragma unroll
-            for (int c = 0; c < 32; ++c)
-              mraw = fmaxf(mraw, (c >= lo && c < hi) ? __uint_as_float(r[c]) : -INFINITY);
+              for (int i = 0; i < 4; ++i) mx[i] = __uint_as_float(r[i]);
+#pragma unroll
+              for (int c = 4; c < 32; ++c) mx[c & 3] = fmaxf(mx[c & 3], __uint_as_float(r[c]));
+              mraw = fmaxf(mraw, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])));
+            } else {
+#pragma unroll
+              for (int c = 0; c < 32; ++c)
+                mraw = fmaxf(mraw, (c >= lo && c < hi) ? __uint_as_float(r[c]) : -INFINITY);
+            }
           }
           mraw = fmaxf(mraw, exchange(mraw));
           if (!both) break;
@@ -446,17 +455,30 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
             tmem_wait_ld_dep32(r);
             uint32_t pk[16];
             const int lo = clo - c0 - cc, hi = chi - c0 - cc;
+            if (lo <= 0 && hi >= 32) {   // warp-uniform: the whole chunk visible
+              float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int c = 0; c < 32; c += 2) {
-              // masked scores enter ex2 as -inf and come out as 0
-              const float x0 = (c >= lo && c < hi) ? fmaf(__uint_as_float(r[c]), p.scale_log2, -mu)
-                                                   : -INFINITY;
-              const float x1 = (c + 1 >= lo && c + 1 < hi)
-                                   ? fmaf(__uint_as_float(r[c + 1]), p.scale_log2, -mu)
-                                   : -INFINITY;
-              const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
-              rs += e0 + e1;
-              pk[c / 2] = pack_bf16x2(e0, e1);
+              for (int c = 0; c < 32; c += 2) {
+                const float2 xx = fma2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])),
+                                       p.scale_log2, -mu);
+                const float2 ee = make_float2(ex2_approx(xx.x), ex2_approx(xx.y));
+                acc = add2(acc, ee);
+                pk[c / 2] = pack_bf16x2(ee.x, ee.y);
+              }
+              rs += acc.x + acc.y;
+            } else {
+#pragma unroll
+              for (int c = 0; c < 32; c += 2) {
+                // masked scores enter ex2 as -inf and come out as 0
+                const float x0 = (c >= lo && c < hi) ? fmaf(__uint_as_float(r[c]), p.scale_log2, -mu)
+                                                     : -INFINITY;
+                const float x1 = (c + 1 >= lo && c + 1 < hi)
+                                     ? fmaf(__uint_as_float(r[c + 1]), p.scale_log2, -mu)
+                                     : -INFINITY;
+                const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
+                rs += e0 + e1;
+                pk[c / 2] = pack_bf16x2(e0, e1);
+              }
             }
             // chunk-major image: 8-key chunk k8 of row `row` at k8 * 2048 + 16 * row
 #pragma unroll

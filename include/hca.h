@@ -216,6 +216,46 @@ hca_status_t hca_decode_step(const hca_bf16* q, const hca_bf16* g, const hca_bf1
                              hca_stream_t stream);
 
 /*
+ * hca_quantize_e4m3 — FP8 storage of 512-wide bf16 rows (e.g. cache entries
+ * and window rows for hca_decode_e4m3).
+ *   The pages train with FP8 mixed precision and ship FP8 weights
+ *   ('BaiduがERNIE 5.5 Flash Baseを公開' §3 and §5); the library stores a
+ *   decode cache the same way.  Per row r:
+ *     scale[r] = amax(|x[r, :]|) / 448            (fp32; 1 for an all-zero row)
+ *     codes[r, c] = e4m3(x[r, c] / scale[r])      (fp32 division, round to
+ *                                                   nearest even, saturating at
+ *                                                   +-448)
+ *   so the stored value is e4m3_value(codes) * scale.
+ * Layout:  x [rows, 512] bf16 (16-byte aligned);  codes [rows, 512] bytes
+ *          (16-byte aligned);  scale [rows] fp32.  Rows must be finite.
+ * Errors:  rows < 0 or a null / misaligned pointer -> HCA_ERR_INVALID_ARG.
+ */
+hca_status_t hca_quantize_e4m3(const hca_bf16* x, long long rows, uint8_t* codes, float* scale,
+                               hca_stream_t stream);
+
+/*
+ * hca_decode_e4m3 — hca_decode over an FP8 cache: the compressed entries and
+ * the raw window rows stored by hca_quantize_e4m3 (half the bytes a decode
+ * step streams).  The result is the HCA decode of the stored values
+ * (code * row scale), as defined for hca_decode; q and g stay bf16, and q must
+ * satisfy |q| < 65504 (the kernel runs its MMAs in f16: every e4m3 value and
+ * every such bf16 value is exact in f16).
+ * Layout:  q, g, out [S, 64, 512] bf16;  ck, cv [S, max_nc, 512] codes with
+ *          ck_scale, cv_scale [S, max_nc] fp32;  wk, wv [S, 128, 512] codes (ring,
+ *          slot = position mod 128) with wk_scale, wv_scale [S, 128] fp32;
+ *          ctx_len [S] int32 on the device;  ws as for hca_decode (the same
+ *          workspace serves both calls).
+ * Errors:  as hca_decode; every scale pointer is required (ck / cv scales only
+ *          when max_nc > 0).
+ */
+hca_status_t hca_decode_e4m3(const hca_bf16* q, const uint8_t* ck, const float* ck_scale,
+                             const uint8_t* cv, const float* cv_scale, int max_nc,
+                             const uint8_t* wk, const float* wk_scale, const uint8_t* wv,
+                             const float* wv_scale, const int32_t* ctx_len, const hca_bf16* g,
+                             int S, int H, float scale, void* ws, size_t ws_bytes, hca_bf16* out,
+                             hca_stream_t stream);
+
+/*
  * hca_get_device_error — synchronises `stream`, then reads and clears the
  * device-side error word of the current device.  Returns HCA_OK,
  * HCA_ERR_TIMEOUT, HCA_ERR_DEVICE_INPUT or HCA_ERR_CUDA.  `where`, if not

@@ -281,6 +281,74 @@ def cache_append(wk, wv, ws, ck, cv, k_new, v_new, s_new, L: int,
 
 
 # ---------------------------------------------------------------------------
+# FP8 (e4m3) cache storage
+# ---------------------------------------------------------------------------
+# The pages train with FP8 mixed precision and ship FP8 weights ('Baiduが
+# ERNIE 5.5 Flash Baseを公開' §3 and §5); the decode cache can be stored the
+# same way.  Reading adopted: every 512-wide cache row is stored as e4m3
+# codes with one fp32 scale, scale = amax(|row|) / 448 (1 for an all-zero
+# row), code = e4m3(row / scale) rounded to nearest even, saturating at the
+# largest finite magnitude 448.  The row's value is code * scale.  The
+# division and the rounding decision are taken in fp32, the precision the
+# kernel takes them in, so both sides produce the same codes.
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """Value of each e4m3 code (1 sign bit, 4 exponent bits with bias 7, 3
+    mantissa bits; exponent field 0 holds subnormals m * 2^-9; 0x7F / 0xFF
+    are NaN; there are no infinities).  Returned as fp64."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * 2.0 ** (e - 7))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return sign * mag
+
+
+def e4m3_encode(y: np.ndarray) -> np.ndarray:
+    """Round each (fp32) value to the nearest e4m3 value, ties to the even
+    mantissa, magnitudes above 448 saturating to 448; NaN -> 0x7F."""
+    y = np.asarray(y, dtype=np.float64)
+    neg = np.signbit(y)
+    a = np.abs(y)
+    nan = np.isnan(a)
+    a = np.where(nan, 0.0, np.minimum(a, E4M3_MAX))
+    # quantum of a's binade: 2^(e - 3) with e = floor(log2 a), at least the
+    # subnormal quantum 2^-9 (binade of 2^-6 and below)
+    _, ex = np.frexp(np.maximum(a, 2.0 ** -6))
+    q = 2.0 ** (ex - 1 - 3)
+    v = np.round(a / q) * q          # numpy rounds halves to even
+    v = np.minimum(v, E4M3_MAX)
+    _, ev = np.frexp(np.where(v > 0, v, 1.0))
+    E = ev - 1 + 7                   # biased exponent of a normal value
+    normal = v >= 2.0 ** -6
+    mant_n = np.where(normal, v / 2.0 ** (ev - 1) * 8 - 8, 0)
+    code = np.where(normal, (E << 3) + mant_n.astype(np.int64),
+                    (v / 2.0 ** -9).astype(np.int64))
+    code = code | np.where(neg, 0x80, 0)
+    code = np.where(nan, 0x7F, code)
+    return code.astype(np.uint8)
+
+
+def quantize_e4m3_rows(x: np.ndarray):
+    """Per-row e4m3 storage of x [..., D]: (codes uint8 [..., D], scale fp32
+    [...]) with scale = amax / 448 in fp32 and codes = e4m3(x / scale), the
+    division in fp32."""
+    x32 = np.asarray(x, dtype=np.float32)
+    amax = np.abs(x32).max(axis=-1)
+    scale = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    y = (x32 / scale[..., None]).astype(np.float32)
+    return e4m3_encode(y), scale
+
+
+def dequantize_e4m3_rows(codes: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """fp64 value of each stored row: code value * row scale."""
+    return e4m3_decode(codes) * np.asarray(scale, dtype=np.float64)[..., None]
+
+
+# ---------------------------------------------------------------------------
 # Work counts (used for FLOP accounting and by the tests)
 # ---------------------------------------------------------------------------
 def visited_pairs(T: int, blk: int = BLOCK, win: int = WINDOW) -> int:

@@ -35,7 +35,7 @@ def test_expected_entry_points_declared():
     names = set(declared_functions())
     for n in ("hca_compress", "hca_prefill_fwd", "hca_decode", "hca_decode_workspace_size",
               "hca_get_device_error", "hca_status_string", "hca_version", "hca_cache_append",
-              "hca_decode_step"):
+              "hca_decode_step", "hca_quantize_e4m3", "hca_decode_e4m3"):
         assert n in names
 
 
@@ -134,6 +134,32 @@ def test_cache_append_and_decode_step_reject_bad_arguments(lib):
     assert step(a15=f + 16) == 1             # workspace not 256-byte aligned
     assert step(a2=None) == 1                # no k_new (append half)
     assert step(a6=70000) == 2               # S beyond what decode supports
+
+
+def test_fp8_entry_points_reject_bad_arguments(lib):
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    f = 1 << 20
+    lib.hca_quantize_e4m3.argtypes = [vp, ctypes.c_longlong, vp, vp, vp]
+    assert lib.hca_quantize_e4m3(f, -1, f, f, None) == 1          # rows < 0
+    assert lib.hca_quantize_e4m3(None, 4, f, f, None) == 1        # no input
+    assert lib.hca_quantize_e4m3(f + 8, 4, f, f, None) == 1       # misaligned input
+    assert lib.hca_quantize_e4m3(f, 4, f, f + 2, None) == 1       # misaligned scales
+    assert lib.hca_quantize_e4m3(None, 0, None, None, None) == 0  # nothing to do
+    lib.hca_decode_e4m3.argtypes = [vp, vp, vp, vp, vp, i, vp, vp, vp, vp, vp, vp, i, i,
+                                    ctypes.c_float, vp, ctypes.c_size_t, vp, vp]
+    base = [f, f, f, f, f, 8, f, f, f, f, f, f, 4, 64, 0.04, f, 1 << 30, f, None]
+
+    def call(**kw):
+        a = list(base)
+        for idx, val in kw.items():
+            a[int(idx[1:])] = val
+        return lib.hca_decode_e4m3(*a)
+    assert call(a13=32) == 2                 # H != 64
+    assert call(a12=0) == 1                  # S < 1
+    assert call(a2=None) == 1                # max_nc > 0 but no ck scale
+    assert call(a7=None) == 1                # no wk scale
+    assert call(a6=f + 4) == 1               # misaligned window codes
+    assert call(a14=float("nan")) == 1       # scale
 
 
 def test_selftest_rejects_bad_limit(lib):
