@@ -29,7 +29,9 @@ the design notes of the repository):
   max(0, t - W + 1) .. t (the window includes the query token itself);
 * one softmax over the union of both key sets, one scale 1/sqrt(D) for all
   keys, no positional encoding, no sink;
-* out = sigmoid(g) * o, elementwise over [T, H, D].
+* out = sigmoid(g) * o, elementwise over [T, H, D];
+* virtual head attention, when asked for, mixes the heads of each position's
+  gated output: y = x + up (down^T x) with down, up [H, r].
 
 Parity status: pinned.  The tests under ``tests/test_oracle_pins.py`` tie
 every function here to something other than itself: a brute-force loop
@@ -125,6 +127,24 @@ def sigmoid(x: np.ndarray) -> np.ndarray:
     return 1.0 / (1.0 + np.exp(-x))
 
 
+def vha_mix(x: np.ndarray, down: np.ndarray, up: np.ndarray) -> np.ndarray:
+    """Virtual head attention: after attention, a light low-rank mix across the
+    heads of one position, with an identity skip ('BaiduがERNIE 5.5 Flash Base
+    を公開' §2.1, virtual head attention; 'ERNIE 5.5 Flash Base 正式发布' §2.1,
+    VHA).  The pages give neither the rank nor where the gate sits; the
+    reading here: the mix acts on the gated output of each position,
+
+        y[h] = x[h] + sum_r up[h, r] * sum_k down[k, r] * x[k],
+
+    x [..., H, D] (heads on the second-to-last axis), down and up [H, r].
+    """
+    x = np.asarray(x, dtype=np.float64)
+    down = np.asarray(down, dtype=np.float64)
+    up = np.asarray(up, dtype=np.float64)
+    z = np.einsum("kr,...kd->...rd", down, x)      # [..., r, D]: the rank-r summary
+    return x + np.einsum("hr,...rd->...hd", up, z)
+
+
 def attend(qrows: np.ndarray, keys: np.ndarray, values: np.ndarray,
            mask: np.ndarray, scale: float):
     """Dense masked softmax attention, all heads sharing one key/value set.
@@ -173,14 +193,16 @@ def prefill_forward(q, k, v, s, g, blk: int = BLOCK, win: int = WINDOW,
                     scale: Optional[float] = None,
                     positions: Optional[Sequence[int]] = None,
                     round_cache_bf16: bool = False, chunk: int = 128,
-                    return_lse: bool = False, cache=None, rows_only: bool = False):
+                    return_lse: bool = False, cache=None, rows_only: bool = False,
+                    vha=None):
     """HCA prefill forward in fp64.
 
     q, g: [B, T, H, D]; k, v: [B, T, D]; s: [B, T].  Returns out [B, T, H, D]
     (or [B, len(positions), H, D] when `positions` selects rows), and the lse
     [.., H] when asked.  With ``rows_only`` q and g hold just the selected rows
     ([B, len(positions), H, D], in the order of `positions`).  `cache` may pass
-    precomputed (cK, cV) from ``compress``.
+    precomputed (cK, cV) from ``compress``.  `vha` = (down, up) applies
+    ``vha_mix`` to the gated output of every position.
     """
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
@@ -210,21 +232,22 @@ def prefill_forward(q, k, v, s, g, blk: int = BLOCK, win: int = WINDOW,
             qr = np.asarray(q[b][rows], dtype=np.float64)
             gr = np.asarray(g[b][rows], dtype=np.float64)
             o, l = _prefill_rows(qr, gr, k[b], v[b], ck[b], cv[b], sel, blk, win, scale)
-            out[b, idx] = o
+            out[b, idx] = o if vha is None else vha_mix(o, *vha)
             lse[b, idx] = l
     return (out, lse) if return_lse else out
 
 
 def decode_forward(q, ck, cv, wk, wv, ctx_len, g, blk: int = BLOCK,
                    win: int = WINDOW, scale: Optional[float] = None,
-                   return_lse: bool = False):
+                   return_lse: bool = False, vha=None):
     """HCA decode for one new token per sequence, in fp64.
 
     q, g: [S, H, D]; ck, cv: [S, max_nc, D]; wk, wv: [S, win, D] hold the
     window as a ring, the token at position p in slot p mod win; ctx_len[s] = L
     counts the new token, so the query sits at t = L - 1.  Keys are the
     compressed entries j < nc(L - 1) and the min(L, win) newest raw tokens
-    (slots 0 .. L-1 when L < win, all slots otherwise).
+    (slots 0 .. L-1 when L < win, all slots otherwise).  `vha` = (down, up)
+    applies ``vha_mix`` to each sequence's gated output.
     """
     q = np.asarray(q, dtype=np.float64)
     g = np.asarray(g, dtype=np.float64)
@@ -247,6 +270,8 @@ def decode_forward(q, ck, cv, wk, wv, ctx_len, g, blk: int = BLOCK,
         mask = np.ones((1, keys.shape[0]), dtype=bool)
         o, l = attend(q[si][None], keys, vals, mask, scale)
         out[si] = sigmoid(g[si]) * o[0]
+        if vha is not None:
+            out[si] = vha_mix(out[si], *vha)
         lse[si] = l[0]
     return (out, lse) if return_lse else out
 
