@@ -49,11 +49,15 @@ def lib() -> ctypes.CDLL:
         vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
         L.hca_compress.argtypes = [vp, vp, vp, i, i, vp, vp, vp]
         L.hca_prefill_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, f, vp, vp, vp, sz, vp]
+        L.hca_prefill_fwd_vha.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, f, vp, vp, i, vp, vp,
+                                          vp, sz, vp]
         L.hca_prefill_workspace_size.argtypes = [i, i]
         L.hca_prefill_workspace_size.restype = sz
         L.hca_decode_workspace_size.argtypes = [i]
         L.hca_decode_workspace_size.restype = sz
         L.hca_decode.argtypes = [vp, vp, vp, i, vp, vp, vp, vp, i, i, f, vp, sz, vp, vp]
+        L.hca_decode_vha.argtypes = [vp, vp, vp, i, vp, vp, vp, vp, i, i, f, vp, vp, i, vp, sz,
+                                     vp, vp]
         L.hca_cache_append.argtypes = [vp, vp, vp, vp, i, vp, vp, vp, vp, vp, i, vp]
         L.hca_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i, i, f, vp, vp, vp, vp, vp, i, vp,
                                       sz, vp, vp]
@@ -67,7 +71,8 @@ def lib() -> ctypes.CDLL:
         L.hca_version.restype = i
         for name in ("hca_compress", "hca_prefill_fwd", "hca_decode", "hca_get_device_error",
                      "hca_selftest_bounded_wait", "hca_cache_append", "hca_decode_step",
-                     "hca_quantize_e4m3", "hca_decode_e4m3"):
+                     "hca_quantize_e4m3", "hca_decode_e4m3", "hca_prefill_fwd_vha",
+                     "hca_decode_vha"):
             getattr(L, name).restype = i
         _LIB = L
     return _LIB
@@ -127,14 +132,26 @@ def prefill_workspace_size(B: int, T: int) -> int:
     return int(lib().hca_prefill_workspace_size(B, T))
 
 
+def _check_vha(vha, device):
+    down, up = vha
+    r = down.shape[1] if down.dim() == 2 else -1
+    _check(down, "vha_down", (HEADS, r))
+    _check(up, "vha_up", (HEADS, r))
+    if not 1 <= r <= HEADS or down.device != device or up.device != device:
+        raise ValueError(f"vha factors must be [64, r] bf16 on {device} with 1 <= r <= 64")
+    return down, up, r
+
+
 def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, ck: torch.Tensor,
             cv: torch.Tensor, g: torch.Tensor, scale: Optional[float] = None,
             out: Optional[torch.Tensor] = None, return_lse: bool = False,
-            workspace: Optional[torch.Tensor] = None):
+            workspace: Optional[torch.Tensor] = None, vha=None):
     """HCA prefill attention with the gate fused.
 
     q, g: [B, T, 64, 512]; k, v: [B, T, 512]; ck, cv: [B, T // 128, 512]
     -> out [B, T, 64, 512] bf16 (and lse [B, T, 64] fp32 when asked).
+    `vha` = (down, up), each [64, r] bf16: virtual head attention fused into
+    the epilogue (hca_prefill_fwd_vha).
     """
     B, T, H, D = q.shape
     _check(q, "q", (B, T, H, HEAD_DIM))
@@ -154,10 +171,19 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, ck: torch.Tensor,
         workspace = torch.empty((prefill_workspace_size(B, T),), dtype=torch.uint8,
                                 device=q.device)
     _check(workspace, "workspace", dtype=torch.uint8)
-    _ok("hca_prefill_fwd", lib().hca_prefill_fwd(
-        q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(ck) if nb else None,
-        _ptr(cv) if nb else None, g.data_ptr(), B, T, H, ctypes.c_float(scale), out.data_ptr(),
-        _ptr(lse), workspace.data_ptr(), workspace.numel(), _stream(q.device)))
+    if vha is None:
+        _ok("hca_prefill_fwd", lib().hca_prefill_fwd(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(ck) if nb else None,
+            _ptr(cv) if nb else None, g.data_ptr(), B, T, H, ctypes.c_float(scale),
+            out.data_ptr(), _ptr(lse), workspace.data_ptr(), workspace.numel(),
+            _stream(q.device)))
+    else:
+        down, up, r = _check_vha(vha, q.device)
+        _ok("hca_prefill_fwd_vha", lib().hca_prefill_fwd_vha(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(ck) if nb else None,
+            _ptr(cv) if nb else None, g.data_ptr(), B, T, H, ctypes.c_float(scale),
+            down.data_ptr(), up.data_ptr(), r, out.data_ptr(), _ptr(lse), workspace.data_ptr(),
+            workspace.numel(), _stream(q.device)))
     return (out, lse) if return_lse else out
 
 
@@ -179,10 +205,12 @@ def decode_workspace(S: int, device) -> torch.Tensor:
 def decode(q: torch.Tensor, ck: torch.Tensor, cv: torch.Tensor, wk: torch.Tensor,
            wv: torch.Tensor, ctx_len: torch.Tensor, g: torch.Tensor,
            scale: Optional[float] = None, workspace: Optional[torch.Tensor] = None,
-           out: Optional[torch.Tensor] = None) -> torch.Tensor:
+           out: Optional[torch.Tensor] = None, vha=None) -> torch.Tensor:
     """One decode step: q, g [S, 64, 512]; ck, cv [S, max_nc, 512]; wk, wv
     [S, 128, 512] ring windows; ctx_len [S] int32 on the device.  A workspace
-    passed in comes from ``decode_workspace`` (zero-filled before first use)."""
+    passed in comes from ``decode_workspace`` (zero-filled before first use).
+    `vha` = (down, up), each [64, r] bf16: virtual head attention fused into
+    the same launch (hca_decode_vha)."""
     S, H, D = q.shape
     _check(q, "q", (S, H, HEAD_DIM))
     _check(g, "g", (S, H, HEAD_DIM))
@@ -200,11 +228,19 @@ def decode(q: torch.Tensor, ck: torch.Tensor, cv: torch.Tensor, wk: torch.Tensor
         out = torch.empty_like(q)
     _check(out, "out", (S, H, HEAD_DIM))
     _check(workspace, "workspace", dtype=torch.uint8)
-    _ok("hca_decode", lib().hca_decode(
-        q.data_ptr(), _ptr(ck) if max_nc else None, _ptr(cv) if max_nc else None, max_nc,
-        wk.data_ptr(), wv.data_ptr(), ctx_len.data_ptr(), g.data_ptr(), S, H,
-        ctypes.c_float(scale), workspace.data_ptr(), workspace.numel(), out.data_ptr(),
-        _stream(q.device)))
+    if vha is None:
+        _ok("hca_decode", lib().hca_decode(
+            q.data_ptr(), _ptr(ck) if max_nc else None, _ptr(cv) if max_nc else None, max_nc,
+            wk.data_ptr(), wv.data_ptr(), ctx_len.data_ptr(), g.data_ptr(), S, H,
+            ctypes.c_float(scale), workspace.data_ptr(), workspace.numel(), out.data_ptr(),
+            _stream(q.device)))
+    else:
+        down, up, r = _check_vha(vha, q.device)
+        _ok("hca_decode_vha", lib().hca_decode_vha(
+            q.data_ptr(), _ptr(ck) if max_nc else None, _ptr(cv) if max_nc else None, max_nc,
+            wk.data_ptr(), wv.data_ptr(), ctx_len.data_ptr(), g.data_ptr(), S, H,
+            ctypes.c_float(scale), down.data_ptr(), up.data_ptr(), r, workspace.data_ptr(),
+            workspace.numel(), out.data_ptr(), _stream(q.device)))
     return out
 
 

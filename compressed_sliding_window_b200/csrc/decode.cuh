@@ -123,6 +123,10 @@ struct Params {
   const float* scv;
   const float* swk;
   const float* swv;
+  // virtual head attention factors [64][vha_rank] bf16 (vha_rank = 0: none)
+  const uint16_t* vha_down;
+  const uint16_t* vha_up;
+  int vha_rank;
 };
 
 __device__ __forceinline__ int nc_of_len(int L) { return L >= 128 ? (L - 128) / 128 : 0; }
@@ -322,6 +326,7 @@ constexpr int kCombItems = 32;             // runs per batch (bounded by the (m,
 constexpr int kCombData = kSmemPT;         // [Q | ring]: 192 KB of partial rows
 constexpr int kCombMl = kSmemPT;           // P^T area: 32 x 512 B of (m, l)
 static_assert(kCombItems * 512 <= 16384, "(m, l) staging area");
+static_assert(4 * kHeads * 64 * 4 <= kSmemPT - kSmemQ, "head-mix buffers");
 
 // sigmoid(g) is held as f16 pairs until the store (its relative rounding,
 // 2^-11, is below that of the bf16 output)
@@ -632,6 +637,76 @@ __device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t& lo, uint32
 // a bf16 pair -> an f16 pair (exact for |x| < 65504 with at most 11 significant bits)
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
   return pack_f16x2(bf16lo_to_f32(w), bf16hi_to_f32(w));
+}
+
+// ---------------------------------------------------------------------------
+// Virtual head attention ('BaiduがERNIE 5.5 Flash Baseを公開' §2.1, VHA):
+// after every CTA's combined rows are in `out` (a second grid barrier), the
+// CTAs mix the 64 heads of each sequence in place, y = x + up (down^T x), one
+// (sequence, 64 value columns) unit at a time: x [64][64] and the factors in
+// fp32 in shared memory, z = down^T x [r][64], then y.  Two small reductions
+// of r x 64 x 64 FMAs per unit, on the CUDA cores.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void vha_load_factors(const Params& p, float* fd, float* fu) {
+  for (int i = threadIdx.x; i < kHeads * p.vha_rank; i += kThreads) {
+    fd[i] = __uint_as_float(static_cast<uint32_t>(p.vha_down[i]) << 16);
+    fu[i] = __uint_as_float(static_cast<uint32_t>(p.vha_up[i]) << 16);
+  }
+}
+
+__device__ __forceinline__ void vha_mix_units(const Params& p, const float* fd, const float* fu,
+                                              float* xs, float* zs) {
+  const int r = p.vha_rank;
+  const int units = p.S * (kDim / 64);
+#pragma unroll 1
+  for (int un = blockIdx.x; un < units; un += gridDim.x) {
+    uint16_t* base = p.out + static_cast<size_t>(un >> 3) * kHeads * kDim + 64 * (un & 7);
+    // written by other CTAs in this launch: plain loads (the barrier acquired them)
+    for (int i = threadIdx.x; i < kHeads * 8; i += kThreads) {
+      const int h = i >> 3, c8 = i & 7;
+      const uint4 w = *reinterpret_cast<const uint4*>(base + h * kDim + 8 * c8);
+      float* d = xs + h * 64 + 8 * c8;
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        d[2 * j] = bf16lo_to_f32(ws[j]);
+        d[2 * j + 1] = bf16hi_to_f32(ws[j]);
+      }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < r * 64; i += kThreads) {   // z[rr][c] = sum_h down[h][rr] x[h][c]
+      const int rr = i >> 6, c = i & 63;
+      float z = 0.f;
+#pragma unroll 8
+      for (int h = 0; h < kHeads; ++h) z = fmaf(fd[h * r + rr], xs[h * 64 + c], z);
+      zs[rr * 64 + c] = z;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < kHeads * 8; i += kThreads) {  // y = x + sum_rr up[h][rr] z[rr]
+      const int h = i >> 3, c8 = i & 7;
+      float y[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) y[j] = xs[h * 64 + 8 * c8 + j];
+#pragma unroll 4
+      for (int rr = 0; rr < r; ++rr) {
+        const float u = fu[h * r + rr];
+        const float4 z0 = *reinterpret_cast<const float4*>(zs + rr * 64 + 8 * c8);
+        const float4 z1 = *reinterpret_cast<const float4*>(zs + rr * 64 + 8 * c8 + 4);
+        y[0] = fmaf(u, z0.x, y[0]);
+        y[1] = fmaf(u, z0.y, y[1]);
+        y[2] = fmaf(u, z0.z, y[2]);
+        y[3] = fmaf(u, z0.w, y[3]);
+        y[4] = fmaf(u, z1.x, y[4]);
+        y[5] = fmaf(u, z1.y, y[5]);
+        y[6] = fmaf(u, z1.z, y[6]);
+        y[7] = fmaf(u, z1.w, y[7]);
+      }
+      *reinterpret_cast<uint4*>(base + h * kDim + 8 * c8) =
+          make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                     pack_bf16x2(y[6], y[7]));
+    }
+    __syncthreads();   // the next unit overwrites xs, zs
+  }
 }
 
 template <bool kF8>
@@ -1181,10 +1256,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   // CTAs merge the partials of their share of the (sequence, head) rows.
   // The partials are read back by bulk copies (the async proxy): every writer
   // orders its generic stores before them.
-  // The arrival counter is never reset: every launch adds exactly gridDim.x
-  // (each CTA arrives once, on every path), so a launch's arrivals fill the
-  // window [k G, (k + 1) G) that the counter's value at its first arrival
-  // falls in, and the barrier is complete when the counter reaches (k + 1) G.
+  // The arrival counter is never reset: every barrier adds exactly gridDim.x
+  // (each CTA arrives once, on every path; a launch with the head mix holds
+  // two barriers, and no CTA arrives at the second before the first is
+  // complete), so a barrier's arrivals fill the window [k G, (k + 1) G) that
+  // the counter's value at its first arrival falls in, and the barrier is
+  // complete when the counter reaches (k + 1) G.
   // It starts at zero (the workspace is zero-filled before first use) and is
   // 64-bit, so it does not wrap.
   __shared__ unsigned long long bar_target;
@@ -1224,6 +1301,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
   combine_cta(p, tiles, gridDim.x, smem, sbase, bar(B_COMB), abort_flag, warp, lane,
               grid_arrive, grid_wait);
+  if (!kF8 && p.vha_rank > 0) {
+    // the combine's buffers are free once every warp is here
+    float* fd = reinterpret_cast<float*>(smem + kSmemQ);   // [64][r]
+    float* fu = fd + kHeads * kHeads;                       // [64][r]
+    float* xs = fu + kHeads * kHeads;                       // [64][64]
+    float* zs = xs + kHeads * 64;                           // [r][64]
+    __syncthreads();
+    vha_load_factors(p, fd, fu);
+    grid_arrive();  // this CTA's rows of out are written (second barrier of the launch)
+    grid_wait();
+    vha_mix_units(p, fd, fu, xs, zs);
+  }
 }
 
 // ---------------------------------------------------------------------------

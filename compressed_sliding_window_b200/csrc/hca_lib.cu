@@ -108,9 +108,10 @@ bool make_map_codes(CUtensorMap* m, const void* base, uint64_t Y, uint64_t Z) {
 }
 
 // How many 4-CTA clusters of the prefill kernel fit on the current device at
-// once.  The shared-memory attribute is a per-device property of the kernel,
-// so it is set, and the occupancy asked, once for every device the process
-// uses (with that device current).
+// once (the smaller answer of its two variants, which share their launch
+// shape).  The shared-memory attribute is a per-device property of each
+// kernel, so it is set, and the occupancy asked, once for every device the
+// process uses (with that device current).
 int prefill_max_clusters() {
   static int cached[kMaxDevices] = {};
   static std::mutex mu;
@@ -119,7 +120,9 @@ int prefill_max_clusters() {
   std::lock_guard<std::mutex> lock(mu);
   if (cached[dev] > 0) return cached[dev];
   namespace P = hca::prefill3;
-  if (cudaFuncSetAttribute(P::prefill3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(P::prefill3_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           P::kSmemAlloc) != cudaSuccess ||
+      cudaFuncSetAttribute(P::prefill3_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            P::kSmemAlloc) != cudaSuccess)
     return -1;
   cudaLaunchConfig_t cfg = {};
@@ -133,9 +136,12 @@ int prefill_max_clusters() {
   attr.val.clusterDim.z = 1;
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, P::prefill3_kernel, &cfg) != cudaSuccess || n <= 0)
+  int n = 0, nv = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, P::prefill3_kernel<false>, &cfg) != cudaSuccess ||
+      cudaOccupancyMaxActiveClusters(&nv, P::prefill3_kernel<true>, &cfg) != cudaSuccess)
     return -1;
+  n = n < nv ? n : nv;
+  if (n <= 0) return -1;
   cached[dev] = n;
   return n;
 }
@@ -225,10 +231,13 @@ size_t hca_prefill_workspace_size(int B, int T) {
   return static_cast<size_t>(clusters) * hca::prefill3::kScratchPerCluster + 256;
 }
 
-hca_status_t hca_prefill_fwd(const hca_bf16* q, const hca_bf16* k, const hca_bf16* v,
-                             const hca_bf16* ck, const hca_bf16* cv, const hca_bf16* g, int B,
-                             int T, int H, float scale, hca_bf16* out, float* lse, void* ws,
-                             size_t ws_bytes, hca_stream_t stream) {
+namespace {
+// hca_prefill_fwd and hca_prefill_fwd_vha (vha_rank = 0: no head mix)
+hca_status_t prefill_impl(const hca_bf16* q, const hca_bf16* k, const hca_bf16* v,
+                          const hca_bf16* ck, const hca_bf16* cv, const hca_bf16* g, int B, int T,
+                          int H, float scale, const hca_bf16* vha_down, const hca_bf16* vha_up,
+                          int vha_rank, hca_bf16* out, float* lse, void* ws, size_t ws_bytes,
+                          cudaStream_t stream) {
   namespace P = hca::prefill3;
   if (H != HCA_NUM_HEADS) return HCA_ERR_UNSUPPORTED;
   if (B < 1 || T < 1 || !scale_ok(scale)) return HCA_ERR_INVALID_ARG;
@@ -274,8 +283,34 @@ hca_status_t hca_prefill_fwd(const hca_bf16* q, const hca_bf16* k, const hca_bf1
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.lse = lse;
   prm.pscratch = static_cast<uint8_t*>(ws);
-  P::prefill3_kernel<<<4 * clusters, P::kThreads, P::kSmemAlloc, stream>>>(maps, prm);
+  prm.vha_down = vha_down;
+  prm.vha_up = vha_up;
+  prm.vha_rank = vha_rank;
+  if (vha_rank > 0)
+    P::prefill3_kernel<true><<<4 * clusters, P::kThreads, P::kSmemAlloc, stream>>>(maps, prm);
+  else
+    P::prefill3_kernel<false><<<4 * clusters, P::kThreads, P::kSmemAlloc, stream>>>(maps, prm);
   return launch_status();
+}
+}  // namespace
+
+hca_status_t hca_prefill_fwd(const hca_bf16* q, const hca_bf16* k, const hca_bf16* v,
+                             const hca_bf16* ck, const hca_bf16* cv, const hca_bf16* g, int B,
+                             int T, int H, float scale, hca_bf16* out, float* lse, void* ws,
+                             size_t ws_bytes, hca_stream_t stream) {
+  return prefill_impl(q, k, v, ck, cv, g, B, T, H, scale, nullptr, nullptr, 0, out, lse, ws,
+                      ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+hca_status_t hca_prefill_fwd_vha(const hca_bf16* q, const hca_bf16* k, const hca_bf16* v,
+                                 const hca_bf16* ck, const hca_bf16* cv, const hca_bf16* g,
+                                 int B, int T, int H, float scale, const hca_bf16* vha_down,
+                                 const hca_bf16* vha_up, int vha_rank, hca_bf16* out, float* lse,
+                                 void* ws, size_t ws_bytes, hca_stream_t stream) {
+  if (vha_rank < 1 || vha_rank > HCA_NUM_HEADS) return HCA_ERR_INVALID_ARG;
+  if (vha_down == nullptr || vha_up == nullptr) return HCA_ERR_INVALID_ARG;
+  return prefill_impl(q, k, v, ck, cv, g, B, T, H, scale, vha_down, vha_up, vha_rank, out, lse,
+                      ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 size_t hca_decode_workspace_size(int S) {
@@ -288,10 +323,15 @@ size_t hca_decode_workspace_size(int S) {
   return 256 + hca::decode::ws_bytes(slots) + 256 + static_cast<size_t>(S + 1) * 8;
 }
 
-hca_status_t hca_decode(const hca_bf16* q, const hca_bf16* ck, const hca_bf16* cv, int max_nc,
-                        const hca_bf16* wk, const hca_bf16* wv, const int32_t* ctx_len,
-                        const hca_bf16* g, int S, int H, float scale, void* ws, size_t ws_bytes,
-                        hca_bf16* out, hca_stream_t stream) {
+}  // extern "C"
+
+namespace {
+// hca_decode and hca_decode_vha (vha_rank = 0: no head mix)
+hca_status_t decode_impl(const hca_bf16* q, const hca_bf16* ck, const hca_bf16* cv, int max_nc,
+                         const hca_bf16* wk, const hca_bf16* wv, const int32_t* ctx_len,
+                         const hca_bf16* g, int S, int H, float scale, const hca_bf16* vha_down,
+                         const hca_bf16* vha_up, int vha_rank, void* ws, size_t ws_bytes,
+                         hca_bf16* out, cudaStream_t stream) {
   namespace D = hca::decode;
   if (H != HCA_NUM_HEADS) return HCA_ERR_UNSUPPORTED;
   if (S < 1 || max_nc < 0 || !scale_ok(scale)) return HCA_ERR_INVALID_ARG;
@@ -323,6 +363,9 @@ hca_status_t hca_decode(const hca_bf16* q, const hca_bf16* ck, const hca_bf16* c
       reinterpret_cast<long long*>(wsb + 256 + ((D::ws_bytes(slots) + 255) & ~size_t(255)));
   prm.g = g;
   prm.out = out;
+  prm.vha_down = vha_down;
+  prm.vha_up = vha_up;
+  prm.vha_rank = vha_rank;
 
   D::Maps maps;
   bool ok = make_map4(&maps.q, q, static_cast<uint64_t>(S) * HCA_NUM_HEADS, 1, 64, 8) &&
@@ -338,6 +381,28 @@ hca_status_t hca_decode(const hca_bf16* q, const hca_bf16* ck, const hca_bf16* c
 
   if (launch_decode<false>(maps, prm, sms, stream) != cudaSuccess) return HCA_ERR_CUDA;
   return launch_status();
+}
+}  // namespace
+
+extern "C" {
+
+hca_status_t hca_decode(const hca_bf16* q, const hca_bf16* ck, const hca_bf16* cv, int max_nc,
+                        const hca_bf16* wk, const hca_bf16* wv, const int32_t* ctx_len,
+                        const hca_bf16* g, int S, int H, float scale, void* ws, size_t ws_bytes,
+                        hca_bf16* out, hca_stream_t stream) {
+  return decode_impl(q, ck, cv, max_nc, wk, wv, ctx_len, g, S, H, scale, nullptr, nullptr, 0, ws,
+                     ws_bytes, out, stream);
+}
+
+hca_status_t hca_decode_vha(const hca_bf16* q, const hca_bf16* ck, const hca_bf16* cv,
+                            int max_nc, const hca_bf16* wk, const hca_bf16* wv,
+                            const int32_t* ctx_len, const hca_bf16* g, int S, int H, float scale,
+                            const hca_bf16* vha_down, const hca_bf16* vha_up, int vha_rank,
+                            void* ws, size_t ws_bytes, hca_bf16* out, hca_stream_t stream) {
+  if (vha_rank < 1 || vha_rank > HCA_NUM_HEADS) return HCA_ERR_INVALID_ARG;
+  if (vha_down == nullptr || vha_up == nullptr) return HCA_ERR_INVALID_ARG;
+  return decode_impl(q, ck, cv, max_nc, wk, wv, ctx_len, g, S, H, scale, vha_down, vha_up,
+                     vha_rank, ws, ws_bytes, out, stream);
 }
 
 }  // extern "C"

@@ -36,6 +36,17 @@
 // entries and one raw tile of 144 keys [t0-127, t0+16] (the window of all four
 // positions, padded to a multiple of 16); P and V move in 128-key sub-tiles.
 //
+// Virtual head attention (kVha; same pages, §2.1, VHA): after the gate, the
+// 64 heads of each position are mixed, y = x + M' x with M' = up down^T
+// (64 x 64, rank r).  It runs in the O pair's epilogue as one more pair MMA
+// per 128-column gate stage, transposed so that the operands already sit
+// where the epilogue leaves them: A = x^T (the gated bf16 stage in shared
+// memory read MN-major: M = 128 value columns per CTA, K = the 64 heads of one
+// position), B = M'^T (each CTA holds 32 of its 64 columns, 4 KB), D = the
+// 128 TMEM columns of O that the stage has just read out (lane = value
+// column, column = head).  The epilogue then adds D to the staged x.  The V
+// ring drops to 4 stages to make room for B.
+//
 // Warp roles (544 threads): warps 0-1 TMA producers, warp 2 TMEM owner and (in
 // even CTAs) MMA issuer, warps 3-10 compute: two warps per TMEM lane quadrant.
 // On S-CTAs each owns one 128-key half of the score rows; on O-CTAs they
@@ -71,9 +82,11 @@ constexpr int kKSlab = 16384;
 // ---- O-CTA shared memory
 constexpr int O_P = 0;             // 2 sub-tile buffers x [16 key chunks][128 rows][8 keys]
 constexpr int kPBuf = 32768;
-constexpr int O_VRING = 65536;     // 5 stages x 2 slabs x [128 keys][64 dv]
+constexpr int O_VRING = 65536;     // 5 stages (4 with VHA) x 2 slabs x [128 keys][64 dv]
 constexpr int kVStages = 5;
+constexpr int kVStagesVha = 4;
 constexpr int kVStage = 32768;
+constexpr int O_VHAB = O_VRING + kVStagesVha * kVStage;   // VHA: [32 heads][64 heads] bf16, SW128
 
 // ---- barriers (every CTA, same offsets)
 constexpr int BAR = 229376;
@@ -83,22 +96,25 @@ enum {
   VFULL = STATSFREE + 1, GFULL = VFULL + kVStages, VEMPTY = GFULL + kVStages,
   PREADY = VEMPTY + kVStages, PFULL = PREADY + 4, PBUFFREE = PFULL + 2, CORR = PBUFFREE + 2,
   PVDONE = CORR + 2, OFULL = PVDONE + 2, OFREE = OFULL + 2, STATSFULL = OFREE + 2,
-  STAGED = STATSFULL + 1, DRAIN = STAGED + 4, NBAR = DRAIN + 1
+  STAGED = STATSFULL + 1, XSTAGED = STAGED + 4, VHADONE = XSTAGED + 4, DRAIN = VHADONE + 4,
+  NBAR = DRAIN + 1
 };
+constexpr int kBarBytes = 640;
 constexpr int kTmemSlot = BAR + 8 * NBAR;
 constexpr int kAbortSlot = kTmemSlot + 4;
 // S-CTA: per-row maxima exchanged by the two warps of a row ([2][2][128]
 // float) and their ok flags ([2][2][4] int)
-constexpr int S_XMAX = BAR + 512;
+constexpr int S_XMAX = BAR + kBarBytes;
 constexpr int S_XOK = S_XMAX + 2048;
 // O-CTA: rescale factors [2 tile parities][128], flags [2][4], 1/l [128]
-constexpr int O_ALPHA = BAR + 512;
+constexpr int O_ALPHA = BAR + kBarBytes;
 constexpr int O_FLAGS = O_ALPHA + 1024;
 constexpr int O_INVL = O_FLAGS + 64;
 constexpr int kSmemBytes = S_XOK + 64;
 constexpr int kSmemAlloc = kSmemBytes;
-static_assert(kAbortSlot + 4 <= BAR + 512, "barrier region overflow");
+static_assert(kAbortSlot + 4 <= BAR + kBarBytes, "barrier region overflow");
 static_assert(O_VRING + kVStages * kVStage <= BAR, "O-CTA ring overflow");
+static_assert(O_VHAB + 4096 <= BAR, "O-CTA VHA operand overflow");
 static_assert(O_INVL + 512 <= kSmemBytes, "O-CTA layout overflow");
 static_assert(S_KRING + kKStages * kKStage <= BAR, "S-CTA layout overflow");
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
@@ -113,6 +129,9 @@ struct Params {
   float scale_log2;  // softmax scale * log2(e)
   float* lse;        // [B, T, 64] or null
   uint8_t* pscratch; // [clusters][2][4][32 KB] P sub-tile images
+  const uint16_t* vha_down;   // VHA factors [64][vha_rank] bf16 (kVha only)
+  const uint16_t* vha_up;
+  int vha_rank;
 };
 
 struct Maps {
@@ -197,8 +216,10 @@ __device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap* map, int x, i
                : "memory");
 }
 
+template <bool kVha>
 __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
     prefill3_kernel(const __grid_constant__ Maps maps, const Params p) {
+  constexpr int NV = kVha ? kVStagesVha : kVStages;   // V ring stages
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sb = smem_u32(smem);
   if ((sb & 1023u) != 0) {  // uniform: every thread sees the same base
@@ -233,8 +254,27 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(bar(OFREE + 1), 8);             // helper warps (value half 1), both O-CTAs
     mbar_init(bar(STATSFULL), 4);
     for (int e = 0; e < 4; ++e) mbar_init(bar(STAGED + e), 4);   // one arrive per epilogue warp
+    for (int e = 0; e < 4; ++e) mbar_init(bar(XSTAGED + e), 8);  // epilogue warps, both O-CTAs
     *abort_flag = 0;
     fence_mbar_init();
+  }
+  if (kVha && isO) {
+    // this CTA's half of B = M'^T: rows n = 32 half + i of M' = up down^T,
+    // K-major (k = input head contiguous), 128B-swizzled, fp32 sums rounded
+    // to bf16
+    for (int idx = threadIdx.x; idx < 32 * 64; idx += kThreads) {
+      const int i = idx >> 6, k = idx & 63;
+      const int n = 32 * half + i;
+      float acc = 0.f;
+      for (int r = 0; r < p.vha_rank; ++r)
+        acc = fmaf(__uint_as_float(static_cast<uint32_t>(p.vha_up[n * p.vha_rank + r]) << 16),
+                   __uint_as_float(static_cast<uint32_t>(p.vha_down[k * p.vha_rank + r]) << 16),
+                   acc);
+      const uint32_t b = pack_bf16x2(acc, 0.f) & 0xFFFFu;
+      *reinterpret_cast<uint16_t*>(smem + O_VHAB + sw128_offset(i, k >> 3) + 2 * (k & 7)) =
+          static_cast<uint16_t>(b);
+    }
+    fence_proxy_async_smem();   // read by the VHA MMAs (async proxy)
   }
   if (warp == 2) {
     tmem_alloc_pair(smem_u32(tmem_slot), 512);
@@ -557,8 +597,8 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
               if ((u & 1) != static_cast<uint32_t>(me)) continue;
               int dh, h;
               pv_stage(s, two, j == 0 || j == x.ntiles - 1, dh, h);
-              const uint32_t st = u % kVStages;
-              ok = mbar_wait(bar(VEMPTY + st), ((u / kVStages) & 1) ^ 1, abort_flag, kWaitLimitNs,
+              const uint32_t st = u % NV;
+              ok = mbar_wait(bar(VEMPTY + st), ((u / NV) & 1) ^ 1, abort_flag, kWaitLimitNs,
                              340);
               if (!ok) break;
               // two 64-column slabs of 128 keys; raw sub-tile 1 is 16 keys: two
@@ -582,8 +622,8 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll 1
           for (int e = 0; e < 4 && ok; ++e, ++u) {   // gate stages of this CTA's rows
             if ((u & 1) != static_cast<uint32_t>(me)) continue;
-            const uint32_t st = u % kVStages;
-            ok = mbar_wait(bar(VEMPTY + st), ((u / kVStages) & 1) ^ 1, abort_flag, kWaitLimitNs,
+            const uint32_t st = u % NV;
+            ok = mbar_wait(bar(VEMPTY + st), ((u / NV) & 1) ^ 1, abort_flag, kWaitLimitNs,
                            341);
             if (!ok) break;
             mbar_expect_tx(bar(GFULL + st), kVStage);
@@ -634,7 +674,7 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
           ubase = gbase + 4;
 #pragma unroll 1
           for (int e = 0; e < 4 && ok; ++e) {
-            const uint32_t st = (gbase + e) % kVStages;
+            const uint32_t st = (gbase + e) % NV;
             ok = mbar_wait(bar(STAGED + e), nitem & 1, abort_flag, kWaitLimitNs, 370);
             if (!ok) break;
             tma_store_4d(&maps.out4, sb + O_VRING + st * kVStage, 0, (x.t0 + orow0) * kHeads,
@@ -644,7 +684,7 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
               // both stages of this value half are in flight: release them as
               // their reads complete
               bulk_wait_read_n<1>();
-              mbar_arrive(bar(VEMPTY + (gbase + e - 1) % kVStages));
+              mbar_arrive(bar(VEMPTY + (gbase + e - 1) % NV));
               bulk_wait_read_all();
               mbar_arrive(bar(VEMPTY + st));
             }
@@ -679,7 +719,7 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
                 ok &= mbar_wait_cluster(bar(OFREE + dh), (nitem & 1) ^ 1, abort_flag, kWaitLimitNs,
                                         352);
               if (dh == 0) ok &= mbar_wait(bar(PFULL + h), sj & 1, abort_flag, kWaitLimitNs, 350);
-              const uint32_t st = u % kVStages;
+              const uint32_t st = u % NV;
               ok &= mbar_wait(bar(VFULL + st), (vpar >> st) & 1, abort_flag, kWaitLimitNs, 353);
               vpar ^= 1u << st;
               tc_fence_after();
@@ -713,6 +753,30 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
           }
           if (!ok) break;
           umma_pair_commit_mc(bar(OFULL + 1), kMaskO);
+          if constexpr (kVha) {
+            // D[c, n] = sum_k x[k, c] M'[n, k] per gate stage and position:
+            // A = the staged x read MN-major (LBO: next 64 value columns,
+            // SBO: next 8 heads), B = M'^T K-major, 4 K steps of 16 heads
+            const uint32_t vdesc = idesc_bf16_f32(2 * kRows, 64, true, false);
+            const uint64_t bd = sdesc_sw128(sb + O_VHAB, 16, 1024);
+#pragma unroll 1
+            for (int e = 0; e < 4 && ok; ++e) {
+              ok &= mbar_wait_cluster(bar(XSTAGED + e), nitem & 1, abort_flag, kWaitLimitNs, 355);
+              if (!ok) break;
+              tc_fence_after();
+              const uint32_t st = (u + e) % NV;
+#pragma unroll
+              for (int pp = 0; pp < 2; ++pp) {
+                const uint64_t ad = sdesc_sw128(sb + O_VRING + st * kVStage + 8192 * pp, 16384, 1024);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                  umma_pair_if(tmem + 128 * e + 64 * pp, ad + 128 * k, bd + 2 * k, vdesc,
+                               k == 0 ? 0u : 1u, true);
+              }
+              umma_pair_commit_mc(bar(VHADONE + e), kMaskO);
+            }
+            if (!ok) break;
+          }
           u += 4;  // gate stages, consumed by the epilogue
         }
         umma_pair_commit_mc(bar(DRAIN), 1u << rank);
@@ -794,14 +858,14 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
         uint32_t gwait = 0;   // bit e: the wait parity of gate stage e
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const uint32_t st = (gbase + e) % kVStages;
+          const uint32_t st = (gbase + e) % NV;
           gwait |= ((gpar >> st) & 1u) << e;
           gpar ^= 1u << st;
         }
 #pragma unroll 1
         for (int e2 = 0; e2 < (helper ? 2 : 1); ++e2) {
           const int e = helper ? 2 + e2 : kv;   // g / out stage: value columns [128e, 128e + 128)
-          const uint32_t st = (gbase + e) % kVStages;
+          const uint32_t st = (gbase + e) % NV;
           if (!mbar_wait_warp(bar(GFULL + st), (gwait >> e) & 1u, abort_flag, kWaitLimitNs, 364)) {
             ok = false;
             break;
@@ -813,7 +877,7 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
             uint32_t o[32];
             tmem_ld32(tq + 128 * e + 32 * q32, o);
             tmem_wait_ld_dep32(o);
-            if (q32 == 3 && e2 == (helper ? 1 : 0)) {  // this warp's part of O read out
+            if (!kVha && q32 == 3 && e2 == (helper ? 1 : 0)) {  // this warp's part of O read out
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive_cluster_relaxed(lbar(OFREE + ee));
@@ -835,8 +899,60 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
             }
           }
           fence_proxy_async_smem();   // this thread's writes, read next by the TMA store
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(STAGED + e));
+          if constexpr (kVha) {       // ... or first by the VHA MMA, which also
+            tc_fence_before();        // overwrites the O columns read above
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(lbar(XSTAGED + e));
+          } else {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(STAGED + e));
+          }
+        }
+        if constexpr (kVha) {
+          // y = x + D: lane = value column c of the stage, D columns = heads.
+          // Lanes c (even) and c + 1 swap one D value per pair of heads
+          // (j, j + 4) so that each writes one bf16 pair: the even lane head
+          // j, the odd lane head j + 4 (rows 4 apart fall on disjoint banks).
+          const int cw = row & ~1;                 // even column of the pair
+          const bool odd = (lane & 1) != 0;
+#pragma unroll 1
+          for (int e2 = 0; e2 < (helper ? 2 : 1) && ok; ++e2) {
+            const int e = helper ? 2 + e2 : kv;
+            const uint32_t st = (gbase + e) % NV;
+            if (!mbar_wait_warp(bar(VHADONE + e), nitem & 1, abort_flag, kWaitLimitNs, 365)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            uint8_t* stage = smem + O_VRING + st * kVStage + (cw >> 6) * 16384;
+#pragma unroll 1
+            for (int i = 0; i < 4; ++i) {          // position i >> 1, heads 32 (i & 1) + 0..31
+              uint32_t d[32];
+              tmem_ld32(tq + 128 * e + 32 * i, d);
+              tmem_wait_ld_dep32(d);
+              if (i == 3 && e2 == (helper ? 1 : 0)) {  // this warp's D read out: O is free
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster_relaxed(lbar(OFREE + ee));
+              }
+              const int r0 = 32 * i + (odd ? 4 : 0);  // stage row of head j (+4 if odd)
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                if (j & 4) continue;
+                const uint32_t send = odd ? d[j] : d[j + 4];
+                const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, 1);
+                const float dl = __uint_as_float(odd ? recv : d[j]);
+                const float dh = __uint_as_float(odd ? d[j + 4] : recv);
+                uint32_t* ptr = reinterpret_cast<uint32_t*>(
+                    stage + sw128_offset(r0 + j, (cw & 63) >> 3) + 2 * (cw & 7));
+                const uint32_t xw = *ptr;
+                *ptr = pack_bf16x2(bf16lo_to_f32(xw) + dl, bf16hi_to_f32(xw) + dh);
+              }
+            }
+            fence_proxy_async_smem();   // read next by the TMA store
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(STAGED + e));
+          }
         }
       }
     }

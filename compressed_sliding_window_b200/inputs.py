@@ -26,7 +26,8 @@ BLOCK = 128
 WINDOW = 128
 CHUNK = 1024
 
-_TENSOR_IDS = {"q": 1, "k": 2, "v": 3, "s": 4, "g": 5, "ck": 6, "cv": 7, "wk": 8, "wv": 9}
+_TENSOR_IDS = {"q": 1, "k": 2, "v": 3, "s": 4, "g": 5, "ck": 6, "cv": 7, "wk": 8, "wv": 9,
+               "vha_down": 10, "vha_up": 11}
 _MASK63 = (1 << 63) - 1
 
 
@@ -184,6 +185,14 @@ def decode_direct_sequence(cfg: DecodeConfig, seq: int, max_nc: int):
     wk = normal_bf16(base, "wk", WINDOW, (HEAD_DIM,))
     wv = normal_bf16(base, "wv", WINDOW, (HEAD_DIM,))
     return ck, cv, wk, wv
+
+
+def vha_factors(rank: int, seed: int, scale: float = 0.125):
+    """Virtual-head-attention factors (down, up), each [64, rank] bf16, drawn
+    N(0, scale^2).  The default 1/8 gives the mixed-in term about sqrt(rank)/8
+    of the size of the gated output."""
+    return (normal_bf16(seed, "vha_down", HEADS, (rank,), scale),
+            normal_bf16(seed, "vha_up", HEADS, (rank,), scale))
 
 
 def decode_query(cfg: DecodeConfig):

@@ -106,6 +106,28 @@ hca_status_t hca_prefill_fwd(const hca_bf16* q, const hca_bf16* k, const hca_bf1
                              size_t ws_bytes, hca_stream_t stream);
 
 /*
+ * hca_prefill_fwd_vha — hca_prefill_fwd followed, inside the same kernel, by
+ *   virtual head attention ('BaiduがERNIE 5.5 Flash Baseを公開' §2.1 and
+ *   'ERNIE 5.5 Flash Base 正式发布' §2.1, VHA: after attention, a light
+ *   low-rank mix across heads with an identity skip, fused into the attention
+ *   kernel at inference).  With x[b, t] the [H, 512] gated output above:
+ *     out[b, t, h, :] = x[h, :] + sum_r up[h, r] * sum_k down[k, r] * x[k, :]
+ *   (the pages give no rank and do not say where the gate sits; this reads
+ *   the mix as acting on the gated output of each position).
+ * Layout:  as hca_prefill_fwd;  vha_down, vha_up [64, vha_rank] bf16
+ *          row-major, device memory, 1 <= vha_rank <= 64.  The mix runs in
+ *          fp32 on bf16 operands: x rounded to bf16 and the 64 x 64 product
+ *          up down^T formed in fp32 and rounded to bf16 once per launch.
+ * Errors:  those of hca_prefill_fwd; HCA_ERR_INVALID_ARG for a rank outside
+ *          [1, 64] or a NULL factor.
+ */
+hca_status_t hca_prefill_fwd_vha(const hca_bf16* q, const hca_bf16* k, const hca_bf16* v,
+                                 const hca_bf16* ck, const hca_bf16* cv, const hca_bf16* g,
+                                 int B, int T, int H, float scale, const hca_bf16* vha_down,
+                                 const hca_bf16* vha_up, int vha_rank, hca_bf16* out, float* lse,
+                                 void* ws, size_t ws_bytes, hca_stream_t stream);
+
+/*
  * hca_decode_workspace_size — bytes of scratch hca_decode needs for S
  * sequences on the current device (partial results of the split-KV pass and
  * a grid-barrier counter).  A workspace must be zero-filled once before its
@@ -139,6 +161,25 @@ hca_status_t hca_decode(const hca_bf16* q, const hca_bf16* ck, const hca_bf16* c
                         const hca_bf16* wk, const hca_bf16* wv, const int32_t* ctx_len,
                         const hca_bf16* g, int S, int H, float scale, void* ws, size_t ws_bytes,
                         hca_bf16* out, hca_stream_t stream);
+
+/*
+ * hca_decode_vha — hca_decode followed, inside the same kernel, by virtual
+ *   head attention on each sequence's gated output (same passage and reading
+ *   as hca_prefill_fwd_vha):
+ *     out[s, h, :] = x[h, :] + sum_r up[h, r] * sum_k down[k, r] * x[k, :]
+ *   with x[s] the [64, 512] output hca_decode would write.  The mix runs in
+ *   fp32 on x rounded to bf16 (a second grid barrier of the launch separates
+ *   the two phases).
+ * Layout:  as hca_decode;  vha_down, vha_up [64, vha_rank] bf16 row-major,
+ *          device memory, 1 <= vha_rank <= 64.
+ * Errors:  those of hca_decode; HCA_ERR_INVALID_ARG for a rank outside
+ *          [1, 64] or a NULL factor.
+ */
+hca_status_t hca_decode_vha(const hca_bf16* q, const hca_bf16* ck, const hca_bf16* cv,
+                            int max_nc, const hca_bf16* wk, const hca_bf16* wv,
+                            const int32_t* ctx_len, const hca_bf16* g, int S, int H, float scale,
+                            const hca_bf16* vha_down, const hca_bf16* vha_up, int vha_rank,
+                            void* ws, size_t ws_bytes, hca_bf16* out, hca_stream_t stream);
 
 /*
  * hca_decode_noalloc — hca_decode for callers that cannot allocate device

@@ -35,7 +35,8 @@ def test_expected_entry_points_declared():
     names = set(declared_functions())
     for n in ("hca_compress", "hca_prefill_fwd", "hca_decode", "hca_decode_workspace_size",
               "hca_get_device_error", "hca_status_string", "hca_version", "hca_cache_append",
-              "hca_decode_step", "hca_quantize_e4m3", "hca_decode_e4m3"):
+              "hca_decode_step", "hca_quantize_e4m3", "hca_decode_e4m3", "hca_prefill_fwd_vha",
+              "hca_decode_vha"):
         assert n in names
 
 
@@ -160,6 +161,41 @@ def test_fp8_entry_points_reject_bad_arguments(lib):
     assert call(a7=None) == 1                # no wk scale
     assert call(a6=f + 4) == 1               # misaligned window codes
     assert call(a14=float("nan")) == 1       # scale
+
+
+def test_vha_entry_points_reject_bad_arguments(lib):
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    f = 1 << 20
+    lib.hca_prefill_fwd_vha.argtypes = [vp] * 6 + [i, i, i, ctypes.c_float, vp, vp, i, vp, vp,
+                                                    vp, ctypes.c_size_t, vp]
+    pre = [f, f, f, f, f, f, 1, 256, 64, 0.04, f, f, 8, f, None, f, 1 << 30, None]
+
+    def prefill(**kw):
+        a = list(pre)
+        for idx, val in kw.items():
+            a[int(idx[1:])] = val
+        return lib.hca_prefill_fwd_vha(*a)
+    assert prefill(a12=0) == 1               # rank < 1
+    assert prefill(a12=65) == 1              # rank > 64
+    assert prefill(a10=None) == 1            # no down factor
+    assert prefill(a11=None) == 1            # no up factor
+    assert prefill(a8=32) == 2               # H != 64
+    assert prefill(a0=None) == 1             # no q
+    lib.hca_decode_vha.argtypes = [vp, vp, vp, i, vp, vp, vp, vp, i, i, ctypes.c_float, vp, vp,
+                                   i, vp, ctypes.c_size_t, vp, vp]
+    dec = [f, f, f, 8, f, f, f, f, 4, 64, 0.04, f, f, 4, f, 1 << 30, f, None]
+
+    def decode(**kw):
+        a = list(dec)
+        for idx, val in kw.items():
+            a[int(idx[1:])] = val
+        return lib.hca_decode_vha(*a)
+    assert decode(a13=0) == 1                # rank < 1
+    assert decode(a13=100) == 1              # rank > 64
+    assert decode(a11=None) == 1             # no down factor
+    assert decode(a12=None) == 1             # no up factor
+    assert decode(a9=32) == 2                # H != 64
+    assert decode(a14=f + 16) == 1           # workspace not 256-byte aligned
 
 
 def test_selftest_rejects_bad_limit(lib):
