@@ -1258,10 +1258,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // orders its generic stores before them.
   // The arrival counter is never reset: every barrier adds exactly gridDim.x
   // (each CTA arrives once, on every path; a launch with the head mix holds
-  // two barriers, and no CTA arrives at the second before the first is
-  // complete), so a barrier's arrivals fill the window [k G, (k + 1) G) that
-  // the counter's value at its first arrival falls in, and the barrier is
-  // complete when the counter reaches (k + 1) G.
+  // two barriers, and every CTA waits for the first to complete before it
+  // arrives at the second -- also a CTA that had no rows to combine and so
+  // never needed the first), so a barrier's arrivals fill the window
+  // [k G, (k + 1) G) that the counter's value at its first arrival falls in,
+  // and the barrier is complete when the counter reaches (k + 1) G.
   // It starts at zero (the workspace is zero-filled before first use) and is
   // 64-bit, so it does not wrap.
   __shared__ unsigned long long bar_target;
@@ -1308,6 +1309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* xs = fu + kHeads * kHeads;                       // [64][64]
     float* zs = xs + kHeads * 64;                           // [r][64]
     __syncthreads();
+    grid_wait();    // the first barrier is complete (a no-op if combining waited for it)
     vha_load_factors(p, fd, fu);
     grid_arrive();  // this CTA's rows of out are written (second barrier of the launch)
     grid_wait();

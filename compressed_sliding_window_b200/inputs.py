@@ -187,10 +187,10 @@ def decode_direct_sequence(cfg: DecodeConfig, seq: int, max_nc: int):
     return ck, cv, wk, wv
 
 
-def vha_factors(rank: int, seed: int, scale: float = 0.125):
+def vha_factors(rank: int, seed: int, scale: float = 1.0 / 16):
     """Virtual-head-attention factors (down, up), each [64, rank] bf16, drawn
-    N(0, scale^2).  The default 1/8 gives the mixed-in term about sqrt(rank)/8
-    of the size of the gated output."""
+    N(0, scale^2).  The default 1/16 (a light mix) makes the mixed-in term
+    about sqrt(rank)/32 of the size of the gated output."""
     return (normal_bf16(seed, "vha_down", HEADS, (rank,), scale),
             normal_bf16(seed, "vha_up", HEADS, (rank,), scale))
 

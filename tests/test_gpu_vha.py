@@ -1,6 +1,17 @@
 """Virtual head attention fused into prefill (hca_prefill_fwd_vha) and decode
 (hca_decode_vha) vs the fp64 oracle, which applies the cross-head mix to the
-gated output of every position.  Every output element is compared."""
+gated output of every position.  Every output element is compared.
+
+Tolerances.  A light mix (factors N(0, 1/16^2): the mixed-in term is at most
+a quarter of the gated output at rank 64) keeps the outputs at the size of
+the plain attention output, and the plain bar applies (max-abs 2e-2,
+relative L2 5e-3).  The kernels mix the gated output as staged in bf16, so
+beside the final bf16 rounding of y each element carries one bf16 rounding
+of x (|x| 2^-9 at most) and the rounding of the mixing matrix (2^-9 of each
+entry): the error bound grows with the output's size.  A strong mix (as large
+as the identity or larger) is therefore held to bars relative to the
+output's largest magnitude: max-abs <= 1e-2 max|y| (2.5 times the 2^-8 max|y|
+that the two roundings reach together) and relative L2 5e-3."""
 import numpy as np
 import pytest
 import torch
@@ -8,7 +19,9 @@ import torch
 import compressed_sliding_window_b200 as hca
 from compressed_sliding_window_b200 import inputs as I
 from oracle import hca_oracle as O
-from tests.gpu_util import assert_close_out, need_gpu, to64
+from tests.gpu_util import OUT_REL_L2, assert_close_out, errors, need_gpu, to64
+
+LIGHT = 1.0 / 16
 
 pytestmark = pytest.mark.gpu
 
@@ -19,7 +32,15 @@ def _check_device():
     assert code == 0, f"device error {code} at {where}"
 
 
-def _prefill_case(B, T, rank, seed, scale=0.125, positions=None):
+def _assert_close_scaled(got, ref, what):
+    assert np.isfinite(got).all(), f"{what}: non-finite values"
+    max_abs, rel = errors(got, ref)
+    top = float(np.abs(ref).max())
+    assert max_abs <= 1e-2 * top and rel <= OUT_REL_L2, \
+        f"{what}: max_abs={max_abs:.3e} (max|y| {top:.3e}) rel_l2={rel:.3e}"
+
+
+def _prefill_case(B, T, rank, seed, scale=LIGHT, positions=None, strong=False):
     cfg = I.PrefillConfig(f"vha{T}", B=B, T=T, seed=seed)
     x = I.prefill_inputs(cfg)
     down, up = I.vha_factors(rank, seed, scale)
@@ -31,7 +52,8 @@ def _prefill_case(B, T, rank, seed, scale=0.125, positions=None):
     if positions is None:
         ref = O.prefill_forward(to64(x["q"]), to64(x["k"]), to64(x["v"]), to64(x["s"]),
                                 to64(x["g"]), vha=vha)
-        assert_close_out(to64(out), ref, f"B={B} T={T} r={rank}")
+        check = _assert_close_scaled if strong else assert_close_out
+        check(to64(out), ref, f"B={B} T={T} r={rank}")
     else:
         ref = O.prefill_forward(to64(x["q"]), to64(x["k"]), to64(x["v"]), to64(x["s"]),
                                 to64(x["g"]), vha=vha, positions=positions)
@@ -49,7 +71,7 @@ def test_prefill_vha_strong_mix_4096():
     """A mix as large as the identity (factor scale 1/2, rank 64) over 4096
     positions: every row."""
     need_gpu()
-    _prefill_case(1, 4096, 64, seed=8200, scale=0.5)
+    _prefill_case(1, 4096, 64, seed=8200, scale=0.5, strong=True)
 
 
 def test_prefill_vha_16k_sampled_rows():
@@ -77,7 +99,7 @@ def test_prefill_vha_matches_plain_kernel_when_mix_is_zero():
     assert torch.equal(plain, mixed)
 
 
-def _decode_case(lens, rank, seed, scale=0.125):
+def _decode_case(lens, rank, seed, scale=LIGHT, strong=False):
     cfg = I.DecodeConfig("vha", S=len(lens), seed=seed, ctx=1, from_raw=False)
     max_nc = max(1, max(max(0, (L - 128) // 128) for L in lens))
     parts = [I.decode_direct_sequence(cfg, i, max_nc) for i in range(len(lens))]
@@ -90,7 +112,8 @@ def _decode_case(lens, rank, seed, scale=0.125):
     _check_device()
     ref = O.decode_forward(to64(q), to64(ck), to64(cv), to64(wk), to64(wv), lens, to64(g),
                            vha=(to64(down), to64(up)))
-    assert_close_out(to64(out), ref, f"lens={lens[:4]} r={rank}")
+    check = _assert_close_scaled if strong else assert_close_out
+    check(to64(out), ref, f"lens={lens[:4]} r={rank}")
 
 
 @pytest.mark.parametrize("lens,rank", [([1], 4), ([5, 127, 128, 129], 1),
@@ -100,6 +123,11 @@ def _decode_case(lens, rank, seed, scale=0.125):
 def test_decode_vha(lens, rank):
     need_gpu()
     _decode_case(lens, rank, seed=8500 + rank + len(lens))
+
+
+def test_decode_vha_strong_mix():
+    need_gpu()
+    _decode_case([3000, 129, 70000, 1], 64, seed=8550, scale=0.5, strong=True)
 
 
 def test_decode_vha_many_sequences():
@@ -118,7 +146,7 @@ def test_decode_vha_long_context_workload():
     parts = [I.decode_direct_sequence(cfg, i, 8191) for i in range(cfg.S)]
     ck, cv, wk, wv = (torch.stack([p[j] for p in parts]) for j in range(4))
     q, g = I.decode_query(cfg)
-    down, up = I.vha_factors(16, 4)
+    down, up = I.vha_factors(16, 4, LIGHT)
     ctx = torch.tensor(lens, dtype=torch.int32, device="cuda")
     out = hca.decode(q.cuda(), ck.cuda(), cv.cuda(), wk.cuda(), wv.cuda(), ctx, g.cuda(),
                      vha=(down.cuda(), up.cuda()))
