@@ -326,7 +326,8 @@ constexpr int kCombItems = 32;             // runs per batch (bounded by the (m,
 constexpr int kCombData = kSmemPT;         // [Q | ring]: 192 KB of partial rows
 constexpr int kCombMl = kSmemPT;           // P^T area: 32 x 512 B of (m, l)
 static_assert(kCombItems * 512 <= 16384, "(m, l) staging area");
-static_assert(4 * kHeads * 64 * 4 <= kSmemPT - kSmemQ, "head-mix buffers");
+static_assert(2 * kHeads * kHeads * 4 + kThreads / 32 * kHeads * 8 * 2 <= kSmemPT - kSmemQ,
+              "head-mix factors and tiles");
 
 // sigmoid(g) is held as f16 pairs until the store (its relative rounding,
 // 2^-11, is below that of the bf16 output)
@@ -642,70 +643,97 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
 // ---------------------------------------------------------------------------
 // Virtual head attention ('BaiduがERNIE 5.5 Flash Baseを公開' §2.1, VHA):
 // after every CTA's combined rows are in `out` (a second grid barrier), the
-// CTAs mix the 64 heads of each sequence in place, y = x + up (down^T x), one
-// (sequence, 64 value columns) unit at a time: x [64][64] and the factors in
-// fp32 in shared memory, z = down^T x [r][64], then y.  Two small reductions
-// of r x 64 x 64 FMAs per unit, on the CUDA cores.
+// warps mix the 64 heads of each sequence in place, y = x + up (down^T x).
+// A warp takes 8 value columns of one sequence: the [64 heads][8] tile comes
+// into its own 1 KB of shared memory with two 16-byte loads per lane; lane
+// (c, q) then holds column c of heads q, q + 4, .., q + 60, forms its part of
+// the rank sums z = down^T x 8 ranks at a time, completes them with two
+// shuffles across the four lanes of its column, and adds up z to its 16
+// accumulators; the tile leaves with 16-byte stores.  Short dependency chains
+// and a small loop body: this code runs once per launch on every warp.  The
+// factors sit in shared memory as fp32, padded with zeros to a multiple of 8
+// ranks.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ int vha_rank8(const Params& p) { return (p.vha_rank + 7) & ~7; }
+
 __device__ __forceinline__ void vha_load_factors(const Params& p, float* fd, float* fu) {
-  for (int i = threadIdx.x; i < kHeads * p.vha_rank; i += kThreads) {
-    fd[i] = __uint_as_float(static_cast<uint32_t>(p.vha_down[i]) << 16);
-    fu[i] = __uint_as_float(static_cast<uint32_t>(p.vha_up[i]) << 16);
+  const int r = p.vha_rank, r8 = vha_rank8(p);
+  for (int i = threadIdx.x; i < kHeads * r8; i += kThreads) {
+    const int h = i / r8, rr = i - h * r8;
+    const bool in = rr < r;
+    fd[i] = in ? __uint_as_float(static_cast<uint32_t>(p.vha_down[h * r + rr]) << 16) : 0.f;
+    fu[i] = in ? __uint_as_float(static_cast<uint32_t>(p.vha_up[h * r + rr]) << 16) : 0.f;
   }
 }
 
-__device__ __forceinline__ void vha_mix_units(const Params& p, const float* fd, const float* fu,
-                                              float* xs, float* zs) {
-  const int r = p.vha_rank;
-  const int units = p.S * (kDim / 64);
+__device__ __forceinline__ void vha_mix_columns(const Params& p, const float* fd, const float* fu,
+                                                uint16_t* tile, int warp, int lane) {
+  const int r8 = vha_rank8(p);
+  const int wpc = kThreads / 32;
+  const int units = p.S * (kDim / 8);
+  const int c = lane & 7, q = lane >> 3;   // this lane: column c, heads q + 4 i (i < 16)
 #pragma unroll 1
-  for (int un = blockIdx.x; un < units; un += gridDim.x) {
-    uint16_t* base = p.out + static_cast<size_t>(un >> 3) * kHeads * kDim + 64 * (un & 7);
+  for (int un = blockIdx.x * wpc + warp; un < units; un += gridDim.x * wpc) {
     // written by other CTAs in this launch: plain loads (the barrier acquired them)
-    for (int i = threadIdx.x; i < kHeads * 8; i += kThreads) {
-      const int h = i >> 3, c8 = i & 7;
-      const uint4 w = *reinterpret_cast<const uint4*>(base + h * kDim + 8 * c8);
-      float* d = xs + h * 64 + 8 * c8;
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    uint16_t* src = p.out + static_cast<size_t>(un >> 6) * kHeads * kDim + 8 * (un & 63);
+    const uint4 a = *reinterpret_cast<const uint4*>(src + lane * kDim);
+    const uint4 b = *reinterpret_cast<const uint4*>(src + (lane + 32) * kDim);
+    *reinterpret_cast<uint4*>(tile + 8 * lane) = a;
+    *reinterpret_cast<uint4*>(tile + 8 * (lane + 32)) = b;
+    __syncwarp();
+    float x[16], y[16];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        d[2 * j] = bf16lo_to_f32(ws[j]);
-        d[2 * j + 1] = bf16hi_to_f32(ws[j]);
+    for (int i = 0; i < 16; ++i) {
+      x[i] = __uint_as_float(static_cast<uint32_t>(tile[(q + 4 * i) * 8 + c]) << 16);
+      y[i] = x[i];
+    }
+#pragma unroll 1
+    for (int r0 = 0; r0 < r8; r0 += 8) {
+      float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {     // this lane's 16 heads of z = down^T x
+        const float* f = fd + (q + 4 * i) * r8 + r0;
+        const float4 fa = *reinterpret_cast<const float4*>(f);
+        const float4 fb = *reinterpret_cast<const float4*>(f + 4);
+        z[0] = fmaf(fa.x, x[i], z[0]);
+        z[1] = fmaf(fa.y, x[i], z[1]);
+        z[2] = fmaf(fa.z, x[i], z[2]);
+        z[3] = fmaf(fa.w, x[i], z[3]);
+        z[4] = fmaf(fb.x, x[i], z[4]);
+        z[5] = fmaf(fb.y, x[i], z[5]);
+        z[6] = fmaf(fb.z, x[i], z[6]);
+        z[7] = fmaf(fb.w, x[i], z[7]);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {      // all 64 heads: the four lanes of column c
+        z[j] += __shfl_xor_sync(0xffffffffu, z[j], 8);
+        z[j] += __shfl_xor_sync(0xffffffffu, z[j], 16);
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {     // y += up z
+        const float* f = fu + (q + 4 * i) * r8 + r0;
+        const float4 fa = *reinterpret_cast<const float4*>(f);
+        const float4 fb = *reinterpret_cast<const float4*>(f + 4);
+        float t = y[i];
+        t = fmaf(fa.x, z[0], t);
+        t = fmaf(fa.y, z[1], t);
+        t = fmaf(fa.z, z[2], t);
+        t = fmaf(fa.w, z[3], t);
+        t = fmaf(fb.x, z[4], t);
+        t = fmaf(fb.y, z[5], t);
+        t = fmaf(fb.z, z[6], t);
+        y[i] = fmaf(fb.w, z[7], t);
       }
     }
-    __syncthreads();
-    for (int i = threadIdx.x; i < r * 64; i += kThreads) {   // z[rr][c] = sum_h down[h][rr] x[h][c]
-      const int rr = i >> 6, c = i & 63;
-      float z = 0.f;
-#pragma unroll 8
-      for (int h = 0; h < kHeads; ++h) z = fmaf(fd[h * r + rr], xs[h * 64 + c], z);
-      zs[rr * 64 + c] = z;
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < kHeads * 8; i += kThreads) {  // y = x + sum_rr up[h][rr] z[rr]
-      const int h = i >> 3, c8 = i & 7;
-      float y[8];
+    __syncwarp();
 #pragma unroll
-      for (int j = 0; j < 8; ++j) y[j] = xs[h * 64 + 8 * c8 + j];
-#pragma unroll 4
-      for (int rr = 0; rr < r; ++rr) {
-        const float u = fu[h * r + rr];
-        const float4 z0 = *reinterpret_cast<const float4*>(zs + rr * 64 + 8 * c8);
-        const float4 z1 = *reinterpret_cast<const float4*>(zs + rr * 64 + 8 * c8 + 4);
-        y[0] = fmaf(u, z0.x, y[0]);
-        y[1] = fmaf(u, z0.y, y[1]);
-        y[2] = fmaf(u, z0.z, y[2]);
-        y[3] = fmaf(u, z0.w, y[3]);
-        y[4] = fmaf(u, z1.x, y[4]);
-        y[5] = fmaf(u, z1.y, y[5]);
-        y[6] = fmaf(u, z1.z, y[6]);
-        y[7] = fmaf(u, z1.w, y[7]);
-      }
-      *reinterpret_cast<uint4*>(base + h * kDim + 8 * c8) =
-          make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
-                     pack_bf16x2(y[6], y[7]));
-    }
-    __syncthreads();   // the next unit overwrites xs, zs
+    for (int i = 0; i < 16; ++i)
+      tile[(q + 4 * i) * 8 + c] = static_cast<uint16_t>(pack_bf16x2(y[i], 0.f) & 0xFFFFu);
+    __syncwarp();
+    *reinterpret_cast<uint4*>(src + lane * kDim) = *reinterpret_cast<const uint4*>(tile + 8 * lane);
+    *reinterpret_cast<uint4*>(src + (lane + 32) * kDim) =
+        *reinterpret_cast<const uint4*>(tile + 8 * (lane + 32));
+    __syncwarp();   // the next unit overwrites the tile
   }
 }
 
@@ -1304,16 +1332,15 @@ __global__ void __launch_bounds__(kThreads, 1)
               grid_arrive, grid_wait);
   if (!kF8 && p.vha_rank > 0) {
     // the combine's buffers are free once every warp is here
-    float* fd = reinterpret_cast<float*>(smem + kSmemQ);   // [64][r]
-    float* fu = fd + kHeads * kHeads;                       // [64][r]
-    float* xs = fu + kHeads * kHeads;                       // [64][64]
-    float* zs = xs + kHeads * 64;                           // [r][64]
+    float* fd = reinterpret_cast<float*>(smem + kSmemQ);   // [64][r8]
+    float* fu = fd + kHeads * kHeads;                       // [64][r8]
+    uint16_t* tiles = reinterpret_cast<uint16_t*>(fu + kHeads * kHeads);   // 1 KB per warp
     __syncthreads();
     grid_wait();    // the first barrier is complete (a no-op if combining waited for it)
     vha_load_factors(p, fd, fu);
     grid_arrive();  // this CTA's rows of out are written (second barrier of the launch)
     grid_wait();
-    vha_mix_units(p, fd, fu, xs, zs);
+    vha_mix_columns(p, fd, fu, tiles + warp * kHeads * 8, warp, lane);
   }
 }
 

@@ -42,10 +42,13 @@
 // per 128-column gate stage, transposed so that the operands already sit
 // where the epilogue leaves them: A = x^T (the gated bf16 stage in shared
 // memory read MN-major: M = 128 value columns per CTA, K = the 64 heads of one
-// position), B = M'^T (each CTA holds 32 of its 64 columns, 4 KB), D = the
-// 128 TMEM columns of O that the stage has just read out (lane = value
-// column, column = head).  The epilogue then adds D to the staged x.  The V
-// ring drops to 4 stages to make room for B.
+// position), B = I then M'^T (two K passes into one accumulator, so the
+// identity term is exact; each CTA holds 32 of the 64 columns of each, 8 KB),
+// D = the 128 TMEM columns of O that the stage has just read out (lane =
+// value column, column = head): D is y itself, which the epilogue rounds and
+// writes over x.  The V ring drops to 4 stages to make room for B.  The mix
+// of value half 1 is issued after the next item's first P.V stages of value
+// half 0, so that waiting for it never holds those back.
 //
 // Warp roles (544 threads): warps 0-1 TMA producers, warp 2 TMEM owner and (in
 // even CTAs) MMA issuer, warps 3-10 compute: two warps per TMEM lane quadrant.
@@ -86,7 +89,7 @@ constexpr int O_VRING = 65536;     // 5 stages (4 with VHA) x 2 slabs x [128 key
 constexpr int kVStages = 5;
 constexpr int kVStagesVha = 4;
 constexpr int kVStage = 32768;
-constexpr int O_VHAB = O_VRING + kVStagesVha * kVStage;   // VHA: [32 heads][64 heads] bf16, SW128
+constexpr int O_VHAB = O_VRING + kVStagesVha * kVStage;   // VHA B: 2 x [32 heads][64 heads] bf16
 
 // ---- barriers (every CTA, same offsets)
 constexpr int BAR = 229376;
@@ -114,7 +117,7 @@ constexpr int kSmemBytes = S_XOK + 64;
 constexpr int kSmemAlloc = kSmemBytes;
 static_assert(kAbortSlot + 4 <= BAR + kBarBytes, "barrier region overflow");
 static_assert(O_VRING + kVStages * kVStage <= BAR, "O-CTA ring overflow");
-static_assert(O_VHAB + 4096 <= BAR, "O-CTA VHA operand overflow");
+static_assert(O_VHAB + 8192 <= BAR, "O-CTA VHA operand overflow");
 static_assert(O_INVL + 512 <= kSmemBytes, "O-CTA layout overflow");
 static_assert(S_KRING + kKStages * kKStage <= BAR, "S-CTA layout overflow");
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
@@ -259,9 +262,9 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (kVha && isO) {
-    // this CTA's half of B = M'^T: rows n = 32 half + i of M' = up down^T,
-    // K-major (k = input head contiguous), 128B-swizzled, fp32 sums rounded
-    // to bf16
+    // this CTA's halves of B: rows n = 32 half + i of the identity and of
+    // M' = up down^T, K-major (k = input head contiguous), 128B-swizzled; M'
+    // as fp32 sums rounded to bf16
     for (int idx = threadIdx.x; idx < 32 * 64; idx += kThreads) {
       const int i = idx >> 6, k = idx & 63;
       const int n = 32 * half + i;
@@ -270,9 +273,10 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
         acc = fmaf(__uint_as_float(static_cast<uint32_t>(p.vha_up[n * p.vha_rank + r]) << 16),
                    __uint_as_float(static_cast<uint32_t>(p.vha_down[k * p.vha_rank + r]) << 16),
                    acc);
-      const uint32_t b = pack_bf16x2(acc, 0.f) & 0xFFFFu;
-      *reinterpret_cast<uint16_t*>(smem + O_VHAB + sw128_offset(i, k >> 3) + 2 * (k & 7)) =
-          static_cast<uint16_t>(b);
+      const uint32_t off = sw128_offset(i, k >> 3) + 2 * (k & 7);
+      *reinterpret_cast<uint16_t*>(smem + O_VHAB + off) = k == n ? 0x3F80u : 0u;   // 1.0, 0
+      *reinterpret_cast<uint16_t*>(smem + O_VHAB + 4096 + off) =
+          static_cast<uint16_t>(pack_bf16x2(acc, 0.f) & 0xFFFFu);
     }
     fence_proxy_async_smem();   // read by the VHA MMAs (async proxy)
   }
@@ -698,6 +702,49 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
         uint32_t u = 0, sj = 0, nitem = 0, ncorr = 0, vpar = 0;
         bool ok = true;
         const uint32_t idesc = idesc_bf16_f32(2 * kRows, 256, false, true);
+        // VHA of gate stages [e0, e1) of the item whose gate stages start at
+        // ring use `gb` (parity `par`): D[c, n] = sum_k x[k, c] (I + M')[n, k]
+        // per position, A = the staged x read MN-major (LBO: next 64 value
+        // columns, SBO: next 8 heads), B = I then M'^T (K-major), 2 x 4 K
+        // steps of 16 heads
+        auto vha_issue = [&](int e0, int e1, uint32_t gb, uint32_t par) -> bool {
+          if constexpr (kVha) {
+            const uint32_t vdesc = idesc_bf16_f32(2 * kRows, 64, true, false);
+            const uint64_t bi = sdesc_sw128(sb + O_VHAB, 16, 1024);
+            const uint64_t bm = sdesc_sw128(sb + O_VHAB + 4096, 16, 1024);
+#pragma unroll 1
+            for (int e = e0; e < e1; ++e) {
+              if (!mbar_wait_cluster(bar(XSTAGED + e), par, abort_flag, kWaitLimitNs, 355))
+                return false;
+              tc_fence_after();
+              const uint32_t st = (gb + e) % NV;
+#pragma unroll
+              for (int pp = 0; pp < 2; ++pp) {
+                const uint64_t ad =
+                    sdesc_sw128(sb + O_VRING + st * kVStage + 8192 * pp, 16384, 1024);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                  umma_pair_if(tmem + 128 * e + 64 * pp, ad + 128 * (k & 3),
+                               (k < 4 ? bi : bm) + 2 * (k & 3), vdesc, k == 0 ? 0u : 1u, true);
+              }
+              umma_pair_commit_mc(bar(VHADONE + e), kMaskO);
+            }
+          }
+          return true;
+        };
+        // value half 1 of the previous item is mixed as soon as its stages
+        // are staged (polled between P.V stages), at the latest before the
+        // first P.V stage of value half 1, whose O columns its D occupies
+        int vha_next = 4;           // next gate stage still to mix (4: none)
+        uint32_t vha_gb = 0, vha_par = 0;
+        auto vha_poll = [&](bool block) -> bool {
+          while (vha_next < 4) {
+            if (!block && !mbar_try_wait_acq_cluster(bar(XSTAGED + vha_next), vha_par)) return true;
+            if (!vha_issue(vha_next, vha_next + 1, vha_gb, vha_par)) return false;
+            ++vha_next;
+          }
+          return true;
+        };
         for (int it = cluster; it < p.items && ok; it += nclusters, ++nitem) {
           const Item x = decode_item(p, it);
           for (int j = 0; j < x.ntiles && ok; ++j, ++sj) {
@@ -715,6 +762,7 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
             for (int s = 0; s < nst; ++s, ++u) {
               int dh, h;
               pv_stage(s, two, first || last, dh, h);
+              if (kVha && vha_next < 4) ok &= vha_poll(first && dh == 1);
               if (first && h == 0)  // this value half of the last item's O is read out
                 ok &= mbar_wait_cluster(bar(OFREE + dh), (nitem & 1) ^ 1, abort_flag, kWaitLimitNs,
                                         352);
@@ -754,31 +802,15 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
           if (!ok) break;
           umma_pair_commit_mc(bar(OFULL + 1), kMaskO);
           if constexpr (kVha) {
-            // D[c, n] = sum_k x[k, c] M'[n, k] per gate stage and position:
-            // A = the staged x read MN-major (LBO: next 64 value columns,
-            // SBO: next 8 heads), B = M'^T K-major, 4 K steps of 16 heads
-            const uint32_t vdesc = idesc_bf16_f32(2 * kRows, 64, true, false);
-            const uint64_t bd = sdesc_sw128(sb + O_VHAB, 16, 1024);
-#pragma unroll 1
-            for (int e = 0; e < 4 && ok; ++e) {
-              ok &= mbar_wait_cluster(bar(XSTAGED + e), nitem & 1, abort_flag, kWaitLimitNs, 355);
-              if (!ok) break;
-              tc_fence_after();
-              const uint32_t st = (u + e) % NV;
-#pragma unroll
-              for (int pp = 0; pp < 2; ++pp) {
-                const uint64_t ad = sdesc_sw128(sb + O_VRING + st * kVStage + 8192 * pp, 16384, 1024);
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                  umma_pair_if(tmem + 128 * e + 64 * pp, ad + 128 * k, bd + 2 * k, vdesc,
-                               k == 0 ? 0u : 1u, true);
-              }
-              umma_pair_commit_mc(bar(VHADONE + e), kMaskO);
-            }
+            ok = vha_issue(0, 2, u, nitem & 1);   // value half 0 now, half 1 polled
             if (!ok) break;
+            vha_next = 2;
+            vha_gb = u;
+            vha_par = nitem & 1;
           }
           u += 4;  // gate stages, consumed by the epilogue
         }
+        if (kVha && ok) ok = vha_poll(true);
         umma_pair_commit_mc(bar(DRAIN), 1u << rank);
         mbar_wait(bar(DRAIN), 0, abort_flag, kWaitLimitNs, 354);
       }
@@ -909,7 +941,7 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
           }
         }
         if constexpr (kVha) {
-          // y = x + D: lane = value column c of the stage, D columns = heads.
+          // y = D: lane = value column c of the stage, D columns = heads.
           // Lanes c (even) and c + 1 swap one D value per pair of heads
           // (j, j + 4) so that each writes one bf16 pair: the even lane head
           // j, the odd lane head j + 4 (rows 4 apart fall on disjoint banks).
@@ -943,10 +975,8 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kThreads, 1)
                 const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, 1);
                 const float dl = __uint_as_float(odd ? recv : d[j]);
                 const float dh = __uint_as_float(odd ? d[j + 4] : recv);
-                uint32_t* ptr = reinterpret_cast<uint32_t*>(
-                    stage + sw128_offset(r0 + j, (cw & 63) >> 3) + 2 * (cw & 7));
-                const uint32_t xw = *ptr;
-                *ptr = pack_bf16x2(bf16lo_to_f32(xw) + dl, bf16hi_to_f32(xw) + dh);
+                *reinterpret_cast<uint32_t*>(stage + sw128_offset(r0 + j, (cw & 63) >> 3) +
+                                             2 * (cw & 7)) = pack_bf16x2(dl, dh);
               }
             }
             fence_proxy_async_smem();   // read next by the TMA store
