@@ -277,6 +277,93 @@ def decode_forward(q, ck, cv, wk, wv, ctx_len, g, blk: int = BLOCK,
 
 
 # ---------------------------------------------------------------------------
+# Backward (training at 128K: 'BaiduがERNIE 5.5 Flash Baseを公開' §3)
+# ---------------------------------------------------------------------------
+def prefill_backward(q, k, v, s, g, dout, blk: int = BLOCK, win: int = WINDOW,
+                     scale: Optional[float] = None, chunk: int = 128):
+    """Gradients of L = sum(dout * out) for out = prefill_forward(q, k, v, s, g).
+
+    Returns dq, dk, dv, ds, dg (the shapes of q, k, v, s, g), in fp64.  The
+    steps follow the forward in reverse, one chunk of query positions at a
+    time over the chunk's union key set with the per-row mask:
+
+      out = sigmoid(g) o            dg = dout o sigmoid(g) (1 - sigmoid(g)),
+                                    dO = dout sigmoid(g)
+      o = P values                  dP = dO . value_j,  dvalue_j += P_j dO
+      P = softmax(z) (masked)       dz = P (dP - sum_j P_j dP_j)
+      z = scale q . key_j           dq = scale sum_j dz_j key_j,
+                                    dkey_j += scale dz_j q
+    Key j is a compressed entry or a raw token; the gradients of the entries
+    then flow through the compressor of each block (softmax weights w of the
+    block's scores):
+      cK = sum_i w_i K_i            dK_i += w_i dcK,  dV_i += w_i dcV
+      w = softmax(s_block)          ds_i = w_i (a_i - sum_m w_m a_m),
+                                    a_i = dcK . K_i + dcV . V_i
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    s = np.asarray(s, dtype=np.float64)
+    g = np.asarray(g, dtype=np.float64)
+    dout = np.asarray(dout, dtype=np.float64)
+    B, T, D = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    ck, cv = compress(k, v, s, blk)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    dg = np.zeros_like(g)
+    dck = np.zeros_like(ck)
+    dcv = np.zeros_like(cv)
+    for b in range(B):
+        for t_lo in range(0, T, chunk):
+            t_hi = min(T, t_lo + chunk) - 1
+            pos = np.arange(t_lo, t_hi + 1)
+            n_c = num_visible_blocks(t_hi, blk, win)
+            r0 = window_start(t_lo, win)
+            keys = np.concatenate([ck[b, :n_c], k[b, r0 : t_hi + 1]], axis=0)
+            vals = np.concatenate([cv[b, :n_c], v[b, r0 : t_hi + 1]], axis=0)
+            raw_idx = np.arange(r0, t_hi + 1)
+            ent_idx = np.arange(n_c)
+            mask = np.zeros((len(pos), n_c + len(raw_idx)), dtype=bool)
+            for row, t in enumerate(pos):
+                t = int(t)
+                mask[row, :n_c] = ent_idx < num_visible_blocks(t, blk, win)
+                mask[row, n_c:] = (raw_idx >= window_start(t, win)) & (raw_idx <= t)
+            qr = q[b, t_lo : t_hi + 1]
+            z = np.einsum("nhd,kd->nhk", qr, keys) * scale
+            z = np.where(mask[:, None, :], z, -np.inf)
+            e = np.exp(z - z.max(axis=-1, keepdims=True))
+            P = e / e.sum(axis=-1, keepdims=True)
+            o = np.einsum("nhk,kd->nhd", P, vals)
+            sg = sigmoid(g[b, t_lo : t_hi + 1])
+            do = dout[b, t_lo : t_hi + 1]
+            dg[b, t_lo : t_hi + 1] = do * o * sg * (1.0 - sg)
+            dO = do * sg
+            dP = np.einsum("nhd,kd->nhk", dO, vals)
+            dz = P * (dP - (P * dP).sum(axis=-1, keepdims=True))
+            dq[b, t_lo : t_hi + 1] = scale * np.einsum("nhk,kd->nhd", dz, keys)
+            dkeys = scale * np.einsum("nhk,nhd->kd", dz, qr)
+            dvals = np.einsum("nhk,nhd->kd", P, dO)
+            dck[b, :n_c] += dkeys[:n_c]
+            dcv[b, :n_c] += dvals[:n_c]
+            dk[b, r0 : t_hi + 1] += dkeys[n_c:]
+            dv[b, r0 : t_hi + 1] += dvals[n_c:]
+    ds = np.zeros_like(s)
+    nb = T // blk
+    for b in range(B):
+        for j in range(nb):
+            sl = slice(j * blk, (j + 1) * blk)
+            w = block_weights(s[b, sl])
+            dk[b, sl] += w[:, None] * dck[b, j]
+            dv[b, sl] += w[:, None] * dcv[b, j]
+            a = k[b, sl] @ dck[b, j] + v[b, sl] @ dcv[b, j]
+            ds[b, sl] = w * (a - (w * a).sum())
+    return dq, dk, dv, ds, dg
+
+
+# ---------------------------------------------------------------------------
 # Incremental cache update (serving)
 # ---------------------------------------------------------------------------
 def cache_append(wk, wv, ws, ck, cv, k_new, v_new, s_new, L: int,
