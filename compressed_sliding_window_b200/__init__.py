@@ -56,6 +56,9 @@ def lib() -> ctypes.CDLL:
         L.hca_decode_workspace_size.argtypes = [i]
         L.hca_decode_workspace_size.restype = sz
         L.hca_decode.argtypes = [vp, vp, vp, i, vp, vp, vp, vp, i, i, f, vp, sz, vp, vp]
+        L.hca_prefill_bwd_workspace_size.argtypes = [i, i]
+        L.hca_prefill_bwd_workspace_size.restype = sz
+        L.hca_prefill_bwd.argtypes = [vp] * 10 + [i, i, i, f] + [vp] * 6 + [sz, vp]
         L.hca_decode_vha.argtypes = [vp, vp, vp, i, vp, vp, vp, vp, i, i, f, vp, vp, i, vp, sz,
                                      vp, vp]
         L.hca_cache_append.argtypes = [vp, vp, vp, vp, i, vp, vp, vp, vp, vp, i, vp]
@@ -72,7 +75,7 @@ def lib() -> ctypes.CDLL:
         for name in ("hca_compress", "hca_prefill_fwd", "hca_decode", "hca_get_device_error",
                      "hca_selftest_bounded_wait", "hca_cache_append", "hca_decode_step",
                      "hca_quantize_e4m3", "hca_decode_e4m3", "hca_prefill_fwd_vha",
-                     "hca_decode_vha"):
+                     "hca_decode_vha", "hca_prefill_bwd"):
             getattr(L, name).restype = i
         _LIB = L
     return _LIB
@@ -185,6 +188,51 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, ck: torch.Tensor,
             down.data_ptr(), up.data_ptr(), r, out.data_ptr(), _ptr(lse), workspace.data_ptr(),
             workspace.numel(), _stream(q.device)))
     return (out, lse) if return_lse else out
+
+
+def prefill_bwd_workspace_size(B: int, T: int) -> int:
+    return int(lib().hca_prefill_bwd_workspace_size(B, T))
+
+
+def prefill_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, s: torch.Tensor,
+                     ck: torch.Tensor, cv: torch.Tensor, g: torch.Tensor, out: torch.Tensor,
+                     lse: torch.Tensor, dout: torch.Tensor, scale: Optional[float] = None,
+                     workspace: Optional[torch.Tensor] = None):
+    """Gradients of sum(dout * out) for the HCA prefill (hca_prefill_bwd).
+
+    q, g, out, dout: [B, T, 64, 512] bf16; k, v: [B, T, 512]; s: [B, T];
+    ck, cv: the forward's compressed cache; lse: [B, T, 64] fp32 from the
+    forward.  Returns dq, dg (bf16, shapes of q and g), dk, dv ([B, T, 512]
+    fp32) and ds ([B, T] fp32) as (dq, dk, dv, ds, dg).
+    """
+    B, T, H, D = q.shape
+    for t, n in ((q, "q"), (g, "g"), (out, "out"), (dout, "dout")):
+        _check(t, n, (B, T, H, HEAD_DIM))
+    _check(k, "k", (B, T, HEAD_DIM))
+    _check(v, "v", (B, T, HEAD_DIM))
+    _check(s, "s", (B, T))
+    nb = T // BLOCK
+    _check(ck, "ck", (B, nb, HEAD_DIM))
+    _check(cv, "cv", (B, nb, HEAD_DIM))
+    _check(lse, "lse", (B, T, H), dtype=torch.float32)
+    if scale is None:
+        scale = 1.0 / math.sqrt(HEAD_DIM)
+    dq = torch.empty_like(q)
+    dg = torch.empty_like(g)
+    dk = torch.empty((B, T, HEAD_DIM), dtype=torch.float32, device=q.device)
+    dv = torch.empty_like(dk)
+    ds = torch.empty((B, T), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty((prefill_bwd_workspace_size(B, T),), dtype=torch.uint8,
+                                device=q.device)
+    _check(workspace, "workspace", dtype=torch.uint8)
+    _ok("hca_prefill_bwd", lib().hca_prefill_bwd(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), s.data_ptr(), _ptr(ck) if nb else None,
+        _ptr(cv) if nb else None, g.data_ptr(), out.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+        B, T, H, ctypes.c_float(scale), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+        ds.data_ptr(), dg.data_ptr(), workspace.data_ptr(), workspace.numel(),
+        _stream(q.device)))
+    return dq, dk, dv, ds, dg
 
 
 def forward(q, k, v, s, g, scale: Optional[float] = None, return_lse: bool = False):

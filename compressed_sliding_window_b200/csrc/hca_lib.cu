@@ -18,6 +18,7 @@
 #include "prefill3.cuh"
 #include "decode.cuh"
 #include "append.cuh"
+#include "backward.cuh"
 #include "quant.cuh"
 
 namespace {
@@ -639,5 +640,157 @@ const char* hca_status_string(hca_status_t status) {
 }
 
 int hca_version(void) { return 100; }
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Backward
+// ---------------------------------------------------------------------------
+namespace {
+
+struct BwdLayout {
+  size_t dO, delta, pc, dsc, pr, dsr, dck, dcv, total;
+  int ncpad;
+};
+
+BwdLayout bwd_layout(int B, int T) {
+  BwdLayout L = {};
+  const size_t rows = static_cast<size_t>(B) * T * HCA_NUM_HEADS;
+  const int nb = T / HCA_BLOCK;
+  L.ncpad = ((nb + 127) / 128) * 128;
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  size_t off = 0;
+  L.dO = off;    off = up(off + rows * HCA_HEAD_DIM * 2);
+  L.delta = off; off = up(off + rows * 4);
+  L.pc = off;    off = up(off + rows * L.ncpad * 2);
+  L.dsc = off;   off = up(off + rows * L.ncpad * 2);
+  L.pr = off;    off = up(off + rows * hca::bwd::kRawW * 2);
+  L.dsr = off;   off = up(off + rows * hca::bwd::kRawW * 2);
+  L.dck = off;   off = up(off + static_cast<size_t>(B) * nb * HCA_HEAD_DIM * 4);
+  L.dcv = off;   off = up(off + static_cast<size_t>(B) * nb * HCA_HEAD_DIM * 4);
+  L.total = off;
+  return L;
+}
+
+// the shared-memory attributes of the backward kernels, once per device
+bool bwd_configured() {
+  static bool done[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done[dev]) return true;
+  namespace W = hca::bwd;
+  if (cudaFuncSetAttribute(W::score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           W::kSmemAllocScore) != cudaSuccess ||
+      cudaFuncSetAttribute(W::dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           W::kSmemAllocGemm) != cudaSuccess ||
+      cudaFuncSetAttribute(W::dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           W::kSmemAllocGemm) != cudaSuccess)
+    return false;
+  done[dev] = true;
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t hca_prefill_bwd_workspace_size(int B, int T) {
+  if (B < 1 || T < 1) return 0;
+  return bwd_layout(B, T).total;
+}
+
+hca_status_t hca_prefill_bwd(const hca_bf16* q, const hca_bf16* k, const hca_bf16* v,
+                             const hca_bf16* s, const hca_bf16* ck, const hca_bf16* cv,
+                             const hca_bf16* g, const hca_bf16* out, const float* lse,
+                             const hca_bf16* dout, int B, int T, int H, float scale, hca_bf16* dq,
+                             float* dk, float* dv, float* ds, hca_bf16* dg, void* ws,
+                             size_t ws_bytes, hca_stream_t stream) {
+  namespace W = hca::bwd;
+  if (H != HCA_NUM_HEADS) return HCA_ERR_UNSUPPORTED;
+  if (B < 1 || T < 1 || !scale_ok(scale)) return HCA_ERR_INVALID_ARG;
+  const void* need[14] = {q, k, v, s, g, out, lse, dout, dq, dk, dv, ds, dg, ws};
+  for (const void* ptr : need)
+    if (ptr == nullptr || !aligned16(ptr)) return HCA_ERR_INVALID_ARG;
+  const int nb = T / HCA_BLOCK;
+  if (nb > 0 && (ck == nullptr || cv == nullptr || !aligned16(ck) || !aligned16(cv)))
+    return HCA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return HCA_ERR_INVALID_ARG;
+  if (static_cast<long long>(T) * HCA_NUM_HEADS > 0x7fffffffLL) return HCA_ERR_UNSUPPORTED;
+  const BwdLayout L = bwd_layout(B, T);
+  if (ws_bytes < L.total) return HCA_ERR_INVALID_ARG;
+  const int sms = device_sms();
+  if (sms <= 0 || !bwd_configured()) return HCA_ERR_CUDA;
+  cudaStream_t st = stream;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+
+  W::Params prm = {};
+  prm.B = B;
+  prm.T = T;
+  prm.nb = nb;
+  prm.ncpad = L.ncpad;
+  prm.ut = (T + 1) / 2;
+  prm.scale = scale;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.dout = dout;
+  prm.out = out;
+  prm.g = g;
+  prm.lse = lse;
+  prm.dO = reinterpret_cast<uint16_t*>(w + L.dO);
+  prm.delta = reinterpret_cast<float*>(w + L.delta);
+  prm.dg = dg;
+  prm.pc = reinterpret_cast<uint16_t*>(w + L.pc);
+  prm.dsc = reinterpret_cast<uint16_t*>(w + L.dsc);
+  prm.pr = reinterpret_cast<uint16_t*>(w + L.pr);
+  prm.dsr = reinterpret_cast<uint16_t*>(w + L.dsr);
+  prm.dq = dq;
+  prm.dk = dk;
+  prm.dv = dv;
+  prm.dck = reinterpret_cast<float*>(w + L.dck);
+  prm.dcv = reinterpret_cast<float*>(w + L.dcv);
+  prm.k = k;
+  prm.v = v;
+  prm.s = s;
+  prm.ds = ds;
+
+  W::Maps maps;
+  const uint64_t rows = static_cast<uint64_t>(T) * HCA_NUM_HEADS;
+  const void* ckb = nb > 0 ? static_cast<const void*>(ck) : static_cast<const void*>(k);
+  const void* cvb = nb > 0 ? static_cast<const void*>(cv) : static_cast<const void*>(v);
+  const uint64_t ny = nb > 0 ? nb : T;
+  const uint64_t ncx = L.ncpad > 0 ? L.ncpad : W::kRawW;
+  const void* pcb = L.ncpad > 0 ? static_cast<const void*>(prm.pc) : prm.pr;
+  const void* dscb = L.ncpad > 0 ? static_cast<const void*>(prm.dsc) : prm.dsr;
+  bool ok = make_map(&maps.q, q, HCA_HEAD_DIM, rows, B, 128) &&
+            make_map(&maps.dO, prm.dO, HCA_HEAD_DIM, rows, B, 128) &&
+            make_map(&maps.ck, ckb, HCA_HEAD_DIM, ny, B, 128) &&
+            make_map(&maps.cv, cvb, HCA_HEAD_DIM, ny, B, 128) &&
+            make_map(&maps.k, k, HCA_HEAD_DIM, T, B, 128) &&
+            make_map(&maps.v, v, HCA_HEAD_DIM, T, B, 128) &&
+            make_map(&maps.dsc_a, dscb, ncx, rows, B, 128) &&
+            make_map(&maps.dsr_a, prm.dsr, W::kRawW, rows, B, 128) &&
+            make_map4(&maps.ck4, ckb, ny, B, 64, 8) && make_map4(&maps.k4, k, T, B, 64, 8) &&
+            make_map(&maps.pc_t, pcb, ncx, rows, B, 64) &&
+            make_map(&maps.dsc_t, dscb, ncx, rows, B, 64) &&
+            make_map(&maps.pr_t, prm.pr, W::kRawW, rows, B, 64) &&
+            make_map(&maps.dsr_t, prm.dsr, W::kRawW, rows, B, 64) &&
+            make_map4(&maps.q4, q, rows, B, 64, 8) && make_map4(&maps.dO4, prm.dO, rows, B, 64, 8);
+  if (!ok) return HCA_ERR_CUDA;
+
+  const size_t nkv = static_cast<size_t>(B) * T * HCA_HEAD_DIM * 4;
+  if (cudaMemsetAsync(dk, 0, nkv, st) != cudaSuccess ||
+      cudaMemsetAsync(dv, 0, nkv, st) != cudaSuccess ||
+      cudaMemsetAsync(ds, 0, static_cast<size_t>(B) * T * 4, st) != cudaSuccess ||
+      (nb > 0 && cudaMemsetAsync(w + L.dck, 0, L.total - L.dck, st) != cudaSuccess))
+    return HCA_ERR_CUDA;
+  const long long nrows = static_cast<long long>(B) * rows;
+  W::prep_kernel<<<static_cast<unsigned>((nrows + 7) / 8), 256, 0, st>>>(prm, nrows);
+  W::score_kernel<<<sms, W::kThreads, W::kSmemAllocScore, st>>>(maps, prm);
+  W::dq_kernel<<<sms, W::kThreads, W::kSmemAllocGemm, st>>>(maps, prm);
+  W::dkv_kernel<<<sms, W::kThreads, W::kSmemAllocGemm, st>>>(maps, prm);
+  if (nb > 0) W::compress_bwd_kernel<<<dim3(nb, B), 128, 0, st>>>(prm);
+  return launch_status();
+}
 
 }  // extern "C"

@@ -27,7 +27,7 @@ WINDOW = 128
 CHUNK = 1024
 
 _TENSOR_IDS = {"q": 1, "k": 2, "v": 3, "s": 4, "g": 5, "ck": 6, "cv": 7, "wk": 8, "wv": 9,
-               "vha_down": 10, "vha_up": 11}
+               "vha_down": 10, "vha_up": 11, "dout": 12}
 _MASK63 = (1 << 63) - 1
 
 

@@ -128,6 +128,44 @@ hca_status_t hca_prefill_fwd_vha(const hca_bf16* q, const hca_bf16* k, const hca
                                  void* ws, size_t ws_bytes, hca_stream_t stream);
 
 /*
+ * hca_prefill_bwd_workspace_size — bytes of device scratch hca_prefill_bwd
+ * needs: dO, the probabilities and their gradients over every visited
+ * (row, key) pair in bf16, and the fp32 entry gradients (about 2 KB per
+ * (position, head) row per 512 compressed entries, plus 1.6 KB per row).
+ * Returns 0 for B < 1 or T < 1.
+ */
+size_t hca_prefill_bwd_workspace_size(int B, int T);
+
+/*
+ * hca_prefill_bwd — gradients of L = sum(dout * out) for out =
+ *   hca_prefill_fwd(q, k, v, hca_compress(k, v, s), g) (the model trains at
+ *   128K context, 'BaiduがERNIE 5.5 Flash Baseを公開' §3).  With o the
+ *   ungated output and P the softmax of each query:
+ *     dg = dout * out * (1 - sigmoid(g)),  dO = dout * sigmoid(g)
+ *     dS = P (dO . value - sum_d dout * out),  dq = scale sum dS key,
+ *     dkey = scale sum dS q,  dvalue = sum P dO  (raw keys and entries),
+ *   and the entry gradients through each block's compressor into dk, dv and
+ *   ds (ds_i = w_i (a_i - sum w a), a_i = dcK . k_i + dcV . v_i).
+ * Layout:  q, g, out, dout, dq, dg [B, T, 64, 512] bf16;  k, v [B, T, 512]
+ *          bf16;  s [B, T] bf16;  ck, cv the forward's [B, T/128, 512];
+ *          lse [B, T, 64] fp32 as written by hca_prefill_fwd;  dk, dv
+ *          [B, T, 512] fp32;  ds [B, T] fp32 (0 for tokens of a partial
+ *          block).  All device memory, 16-byte aligned; ws 256-byte aligned,
+ *          at least hca_prefill_bwd_workspace_size(B, T) bytes, contents
+ *          meaningless before and after.  Five launches on `stream`.
+ * Errors:  HCA_ERR_UNSUPPORTED for H != 64 or T * 64 >= 2^31;
+ *          HCA_ERR_INVALID_ARG for a NULL or misaligned pointer, B, T < 1, a
+ *          non-finite or non-positive scale, or a short workspace;
+ *          HCA_ERR_CUDA for a launch failure.
+ */
+hca_status_t hca_prefill_bwd(const hca_bf16* q, const hca_bf16* k, const hca_bf16* v,
+                             const hca_bf16* s, const hca_bf16* ck, const hca_bf16* cv,
+                             const hca_bf16* g, const hca_bf16* out, const float* lse,
+                             const hca_bf16* dout, int B, int T, int H, float scale, hca_bf16* dq,
+                             float* dk, float* dv, float* ds, hca_bf16* dg, void* ws,
+                             size_t ws_bytes, hca_stream_t stream);
+
+/*
  * hca_decode_workspace_size — bytes of scratch hca_decode needs for S
  * sequences on the current device (partial results of the split-KV pass and
  * a grid-barrier counter).  A workspace must be zero-filled once before its

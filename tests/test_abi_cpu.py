@@ -36,7 +36,7 @@ def test_expected_entry_points_declared():
     for n in ("hca_compress", "hca_prefill_fwd", "hca_decode", "hca_decode_workspace_size",
               "hca_get_device_error", "hca_status_string", "hca_version", "hca_cache_append",
               "hca_decode_step", "hca_quantize_e4m3", "hca_decode_e4m3", "hca_prefill_fwd_vha",
-              "hca_decode_vha"):
+              "hca_decode_vha", "hca_prefill_bwd", "hca_prefill_bwd_workspace_size"):
         assert n in names
 
 
@@ -196,6 +196,36 @@ def test_vha_entry_points_reject_bad_arguments(lib):
     assert decode(a12=None) == 1             # no up factor
     assert decode(a9=32) == 2                # H != 64
     assert decode(a14=f + 16) == 1           # workspace not 256-byte aligned
+
+
+def test_backward_rejects_bad_arguments(lib):
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    f = 1 << 20
+    lib.hca_prefill_bwd.argtypes = [vp] * 10 + [i, i, i, ctypes.c_float] + [vp] * 6 + \
+        [ctypes.c_size_t, vp]
+    base = [f] * 10 + [1, 300, 64, 0.04] + [f] * 6 + [1 << 40, None]
+
+    def call(**kw):
+        a = list(base)
+        for idx, val in kw.items():
+            a[int(idx[1:])] = val
+        return lib.hca_prefill_bwd(*a)
+    assert call(a12=32) == 2                 # H != 64
+    assert call(a10=0) == 1                  # B < 1
+    assert call(a11=0) == 1                  # T < 1
+    assert call(a13=float("inf")) == 1       # scale
+    assert call(a0=None) == 1                # no q
+    assert call(a8=None) == 1                # no lse
+    assert call(a4=None) == 1                # T = 300 has entries but no ck
+    assert call(a14=f + 4) == 1              # misaligned dq
+    assert call(a19=f + 16) == 1             # workspace not 256-byte aligned
+    assert call(a20=1024) == 1               # workspace too small
+    lib.hca_prefill_bwd_workspace_size.argtypes = [i, i]
+    lib.hca_prefill_bwd_workspace_size.restype = ctypes.c_size_t
+    assert lib.hca_prefill_bwd_workspace_size(0, 10) == 0
+    small = lib.hca_prefill_bwd_workspace_size(1, 128)
+    big = lib.hca_prefill_bwd_workspace_size(1, 256)
+    assert 0 < small < big
 
 
 def test_selftest_rejects_bad_limit(lib):
