@@ -3,10 +3,14 @@ gradient).
 
 Tolerance, derived from the arithmetic: the kernels hold P, dS and dO in
 bf16 (relative rounding 2^-9 each) and accumulate in fp32; the forward's
-output and compressed cache they start from are bf16 as well.  Every
-gradient element is a sum of such products, so its relative error is a few
-times 2^-9 ~ 2e-3: the bar is relative L2 <= 1e-2 and max-abs <= 2e-2 of the
-largest magnitude of that gradient.
+output and compressed cache they start from are bf16 as well.  dS = P (dP -
+D) subtracts two roundings of nearly the same number (dP = bf16(dO) . v,
+D = sum dout * out), so its error is about 2^-8 of P |dP| rather than of
+|dS|; in a row with n visible keys dP - D keeps sqrt(1 - 1/n) of the spread
+of dP, hence a relative error of at most 2^-8 sqrt(2) for n >= 2, plus 2^-8
+from the operand roundings: about 1e-2 in the worst case (sequences of two
+or three tokens), a few times 2^-9 for long ones.  The bar is relative L2
+<= 2e-2 and max-abs <= 2e-2 of the largest magnitude of each gradient.
 
 One exception: a single token sees a single key, its softmax is constant and
 the exact dq and dk are 0.  The kernel's dS there is dP - D with
@@ -50,29 +54,45 @@ def _run(B, T, seed, q_scale=1.0):
     return x, dout, [to64(t) for t in grads], ref
 
 
+def _single_key_dq_bound(x, dout, b):
+    """Per-element bound on dq at position 0 of sequence b (one key: the exact
+    value is 0; see the module docstring)."""
+    g = to64(x["g"])[b, 0]
+    dO = to64(dout)[b, 0] / (1.0 + np.exp(-g))
+    v, k = to64(x["v"])[b, 0], to64(x["k"])[b, 0]
+    ds_bound = 2.0 ** -7 * np.linalg.norm(dO, axis=1) * np.linalg.norm(v)
+    return ds_bound[:, None] * np.abs(k)[None, :] / np.sqrt(512.0)
+
+
 def _case(B, T, seed, q_scale=1.0):
-    _, _, grads, ref = _run(B, T, seed, q_scale)
+    x, dout, grads, ref = _run(B, T, seed, q_scale)
+    # position 0 sees one key: its dq is checked against the single-key bound,
+    # the other positions against the relative bars
+    for b in range(B):
+        assert (np.abs(grads[0][b, 0]) <= _single_key_dq_bound(x, dout, b)).all()
+    grads[0], ref = grads[0][:, 1:], [ref[0][:, 1:]] + list(ref[1:])
     for name, got, want in zip(NAMES, grads, ref):
         assert np.isfinite(got).all(), f"{name}: non-finite values"
         max_abs, rel = errors(got, want)
         top = float(np.abs(want).max())
-        assert rel <= 1e-2 and max_abs <= 2e-2 * max(top, 1e-30), \
+        print(f"B={B} T={T} {name}: max_abs={max_abs:.3e} (max {top:.3e}) rel_l2={rel:.3e}")
+        assert rel <= 2e-2 and max_abs <= 2e-2 * max(top, 1e-30), \
             f"B={B} T={T} {name}: max_abs={max_abs:.3e} (max {top:.3e}) rel_l2={rel:.3e}"
 
 
 def test_backward_single_token():
     need_gpu()
     x, dout, (dq, dk, dv, ds, dg), ref = _run(1, 1, seed=9001)
-    q, k, v, g = to64(x["q"])[0, 0], to64(x["k"])[0, 0], to64(x["v"])[0, 0], to64(x["g"])[0, 0]
+    q, v, g = to64(x["q"])[0, 0], to64(x["v"])[0, 0], to64(x["g"])[0, 0]
     dO = to64(dout)[0, 0] / (1.0 + np.exp(-g))                       # [64, 512]
     scale = 1.0 / np.sqrt(512.0)
     ds_bound = 2.0 ** -7 * np.linalg.norm(dO, axis=1) * np.linalg.norm(v)   # [64]
-    assert (np.abs(dq[0, 0]) <= scale * ds_bound[:, None] * np.abs(k)[None, :]).all()
+    assert (np.abs(dq[0, 0]) <= _single_key_dq_bound(x, dout, 0)).all()
     assert (np.abs(dk[0, 0]) <= scale * ds_bound.max() * np.abs(q).sum(0)).all()
     assert not ds.any()                                               # no complete block
     for name, got, want in (("dv", dv, ref[2]), ("dg", dg, ref[4])):
         max_abs, rel = errors(got, want)
-        assert rel <= 1e-2 and max_abs <= 2e-2 * np.abs(want).max(), (name, max_abs, rel)
+        assert rel <= 2e-2 and max_abs <= 2e-2 * np.abs(want).max(), (name, max_abs, rel)
 
 
 @pytest.mark.parametrize("B,T", [(1, 2), (1, 5), (1, 127), (1, 128), (1, 129), (1, 254),
