@@ -487,7 +487,10 @@ def run_ours(args):
                      "ms_per_step": e2e_ms / args.e2e_steps}
     if rank == 0 and not args.quick:
         result["vha"] = bench_prefill_vha(d, ck, cv, out, ws, flops, prefill_ms, dev, peaks, args)
-    del d, out, hout, x, hx, ck, cv, ws
+    del hout, x, hx, ws
+    if rank == 0 and not args.quick:
+        result["backward"] = bench_backward(cfg, d, ck, cv, dev, peaks, args)
+    del d, out, ck, cv
     torch.cuda.empty_cache()
 
     if rank == 0 and not args.quick:
@@ -550,6 +553,71 @@ def bench_prefill_vha(d, ck, cv, out, ws, flops, plain_ms, dev, peaks, args):
                          "frac": (flops + vha_flops) / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
                          "peak_source": peaks["source"] + " (bf16 dense, burst)"},
             "timing": f"CUDA events around each of {n} launches"}
+
+
+def backward_bytes(B: int, T: int) -> int:
+    """HBM bytes the five-pass backward moves at the least, in units of one
+    [B, T, 64, 512] bf16 activation: prep reads dout, out, g and writes dO, dg
+    (5); the score pass reads q and dO (2); dq is written (1); the dK/dV pass
+    reads q and dO (2).  P and dS over every visited (row, key) pair in bf16:
+    written once each, P read once (dV) and dS twice (dq, dK).  dk, dv fp32."""
+    act = B * T * 64 * 512 * 2
+    pairs = B * visited_pairs(T) * 64
+    return 10 * act + 5 * pairs * 2 + 2 * B * T * 512 * 4
+
+
+def bench_backward(cfg, d, ck, cv, dev, peaks, args):
+    """hca_prefill_bwd on the headline workload (T = 131072): CUDA events
+    around each call (five launches), inputs resident."""
+    import torch
+    import compressed_sliding_window_b200 as hca
+    from compressed_sliding_window_b200 import inputs as I
+    B, T = cfg.B, cfg.T
+    out, lse = hca.prefill(d["q"], d["k"], d["v"], ck, cv, d["g"], return_lse=True)
+    dout = torch.empty_like(out)
+    for c in range(0, B * T, 8192):   # N(0, 1) upstream gradient, drawn on the device
+        n = min(8192, B * T - c)
+        dout.view(B * T, 64, 512)[c:c + n] = torch.randn(
+            (n, 64, 512), generator=torch.Generator(dev).manual_seed(c + 7), device=dev,
+            dtype=torch.float32).to(torch.bfloat16)
+    ws = torch.empty((hca.prefill_bwd_workspace_size(B, T),), dtype=torch.uint8, device=dev)
+
+    def call():
+        return hca.prefill_backward(d["q"], d["k"], d["v"], d["s"], ck, cv, d["g"], out, lse,
+                                    dout, workspace=ws)
+    call()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    n = max(3, args.side_steps // 4)
+    times = []
+    for _ in range(n):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        call()
+        b.record(stream)
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    code, where = hca.device_error(dev)
+    if code != 0:
+        raise RuntimeError(f"device error {code} at {where} (backward)")
+    ms = statistics.median(times)
+    flops = 5 * B * visited_pairs(T) * FLOP_PER_PAIR // 2   # S, dP, dq, dk, dv
+    alg = backward_bytes(B, T)
+    del out, lse, dout, ws
+    torch.cuda.empty_cache()
+    return {"workload": f"HCA prefill backward, B={B} T={T} (dq, dk, dv, ds, dg)",
+            "ms_per_call": ms, "launches_per_call": 5, "algorithmic_flops": flops,
+            "roofline": {"bound": "tensor", "achieved": flops / (ms / 1e3) / 1e12,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+                         "peak_source": peaks["source"] + " (bf16 dense, burst)"},
+            "design_traffic": {"bytes": alg, "achieved": alg / (ms / 1e3) / 1e9,
+                               "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                               "frac": alg / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                               "note": "least HBM bytes of this five-pass design (P and dS "
+                                       "go through HBM), not of the method"},
+            "timing": f"CUDA events around each of {n} calls, median"}
 
 
 def bench_prefill_side(cfg, dev, peaks, args):
@@ -732,7 +800,8 @@ def bench_decode(cfg, dev, peaks, args):
 
 def run_profile_case(args):
     """A few launches of one kernel family on a small synthetic case, for ncu
-    captures (--profile-case prefill:T or decode:S:L).  Inputs are drawn on the
+    captures (--profile-case prefill:T, decode:S:L, decode-long[:fp8] or
+    backward:T).  Inputs are drawn on the
     device; nothing is timed or printed but a status line."""
     import torch
     import compressed_sliding_window_b200 as hca
@@ -769,6 +838,14 @@ def run_profile_case(args):
         ctx = torch.full((S,), L, dtype=torch.int32, device=dev)
         for _ in range(args.warmup):
             hca.decode(q, ck, cv, wk, wv, ctx, gg)
+    elif kind == "backward":
+        T = int(dims[0])
+        q, gg, k, v, s = rnd(1, T, 64, 512), rnd(1, T, 64, 512), rnd(1, T, 512), rnd(1, T, 512), rnd(1, T)
+        dout = rnd(1, T, 64, 512)
+        ck, cv = hca.compress(k, v, s)
+        out, lse = hca.prefill(q, k, v, ck, cv, gg, return_lse=True)
+        for _ in range(args.warmup):
+            hca.prefill_backward(q, k, v, s, ck, cv, gg, out, lse, dout)
     else:
         raise SystemExit(f"unknown profile case {args.profile_case}")
     torch.cuda.synchronize()

@@ -53,3 +53,14 @@ def test_compress_bytes():
     assert bench.compress_bytes(1, 131072) == 1024 * (2 * 128 * 512 * 2 + 128 * 2 + 2 * 512 * 2)
     assert bench.compress_bytes(1, 131072) == 1024 * 264448
     assert bench.compress_bytes(2, 300) == 2 * 2 * 264448    # the ragged tail is not read
+
+
+def test_backward_accounting():
+    """Five pair-GEMMs (S, dP, dq, dk, dv) against the forward's two; the
+    design's least bytes at T = 131072 (10 activations + 5 passes over P/dS)."""
+    import bench
+    T = 131072
+    pairs = bench.visited_pairs(T)
+    assert 5 * pairs * bench.FLOP_PER_PAIR // 2 == 5 * pairs * 64 * 512 * 2
+    act = T * 64 * 512 * 2
+    assert bench.backward_bytes(1, T) == 10 * act + 5 * pairs * 64 * 2 + 2 * T * 512 * 4
