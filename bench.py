@@ -485,22 +485,40 @@ def run_ours(args):
     result["e2e"] = {"value": job_throughput(flops, world, args.e2e_steps, e2e_ms) / 1e12,
                      "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                      "ms_per_step": e2e_ms / args.e2e_steps}
-    if rank == 0 and not args.quick:
-        result["vha"] = bench_prefill_vha(d, ck, cv, out, ws, flops, prefill_ms, dev, peaks, args)
-    del hout, x, hx, ws
-    if rank == 0 and not args.quick:
-        result["backward"] = bench_backward(cfg, d, ck, cv, dev, peaks, args)
-    del d, out, ck, cv
-    torch.cuda.empty_cache()
+    # Side measurements after the headline.  A failure in one of them is
+    # recorded in the line (the CUDA context may then be unusable, so the
+    # remaining GPU entries are skipped) instead of losing the headline.
+    side_ok = True
+
+    def side(key, fn):
+        nonlocal side_ok
+        if not side_ok:
+            return
+        try:
+            result[key] = fn()
+        except Exception as e:  # noqa: BLE001
+            side_ok = False
+            result.setdefault("side_errors", {})[key] = f"{type(e).__name__}: {e}"[:300]
 
     if rank == 0 and not args.quick:
-        result["prefill_32k"] = bench_prefill_side(I.PREFILL_32K, dev, peaks, args)
-        result["decode"] = [bench_decode(I.DECODE_64x128K, dev, peaks, args),
-                            bench_decode(I.DECODE_16xLONG, dev, peaks, args)]
+        side("vha", lambda: bench_prefill_vha(d, ck, cv, out, ws, flops, prefill_ms, dev, peaks,
+                                              args))
+    del hout, x, hx, ws
+    if rank == 0 and not args.quick:
+        side("backward", lambda: bench_backward(cfg, d, ck, cv, dev, peaks, args))
+    del d, out, ck, cv
+    if side_ok:
+        torch.cuda.empty_cache()
+
+    if rank == 0 and not args.quick:
+        side("prefill_32k", lambda: bench_prefill_side(I.PREFILL_32K, dev, peaks, args))
+        side("decode", lambda: [bench_decode(I.DECODE_64x128K, dev, peaks, args),
+                                bench_decode(I.DECODE_16xLONG, dev, peaks, args)])
     if rank == 0 and world == 1 and not args.no_cpu:
         result["cpu_baseline"] = cpu_baseline_prefill(cfg)
-        if not args.quick:
+        if not args.quick and "prefill_32k" in result:
             result["prefill_32k"]["cpu_baseline"] = cpu_baseline_prefill(I.PREFILL_32K)
+        if not args.quick and "decode" in result:
             result["decode"][0]["cpu_baseline"] = cpu_baseline_decode(I.DECODE_64x128K, 1024,
                                                                       n_seq=host_cores())
             result["decode"][1]["cpu_baseline"] = cpu_baseline_decode(I.DECODE_16xLONG, 8191)
