@@ -178,7 +178,7 @@ def _f64(t):
     return t.float().numpy().astype(np.float64)
 
 
-def _prefill_worker_init(cfg):
+def _prefill_worker_init(cfg, vha_rank=None):
     import torch
     torch.set_num_threads(1)
     from compressed_sliding_window_b200 import inputs as I
@@ -187,7 +187,8 @@ def _prefill_worker_init(cfg):
     k = _f64(I.normal_bf16(base, "k", cfg.T, (512,), scale=cfg.k_scale))[None]
     v = _f64(I.normal_bf16(base, "v", cfg.T, (512,)))[None]
     s = _f64(I.normal_bf16(base, "s", cfg.T, ()))[None]
-    _CW.update(cfg=cfg, k=k, v=v, s=s, cache=O.compress(k, v, s), base=base)
+    vha = None if vha_rank is None else tuple(_f64(t) for t in I.vha_factors(vha_rank, 1))
+    _CW.update(cfg=cfg, k=k, v=v, s=s, cache=O.compress(k, v, s), base=base, vha=vha)
 
 
 def _prefill_worker_group(job):
@@ -205,7 +206,7 @@ def _prefill_worker_group(job):
     pos = list(range(t0, t0 + q.shape[1]))
     t = time.perf_counter()
     O.prefill_forward(q, _CW["k"], _CW["v"], _CW["s"], g, positions=pos, rows_only=True,
-                      cache=_CW["cache"])
+                      cache=_CW["cache"], vha=_CW["vha"])
     return time.perf_counter() - t, sum(nc_of(x) + min(x + 1, WINDOW) for x in pos) * FLOP_PER_PAIR
 
 
@@ -223,7 +224,7 @@ def time_oracle_compress(cfg) -> float:
     return time.perf_counter() - t
 
 
-def cpu_baseline_prefill(cfg, groups_per_core=2):
+def cpu_baseline_prefill(cfg, groups_per_core=2, vha_rank=None):
     """Oracle TFLOP/s for compress + prefill of `cfg`: every core runs
     oracle groups of 128 consecutive positions, the groups spread evenly over
     the sequence; the rate of all cores together (each core's FLOPs over its
@@ -233,7 +234,7 @@ def cpu_baseline_prefill(cfg, groups_per_core=2):
     T = cfg.T
     n = host_cores()
     starts = [int(x) // BLOCK * BLOCK for x in np.linspace(0, T - BLOCK, n * groups_per_core)]
-    pool = _cpu_pool(n, _prefill_worker_init, (cfg,))
+    pool = _cpu_pool(n, _prefill_worker_init, (cfg, vha_rank))
     try:
         res = pool.map(_prefill_worker_group, [(t0, BLOCK) for t0 in starts], chunksize=1)
     finally:
@@ -244,11 +245,46 @@ def cpu_baseline_prefill(cfg, groups_per_core=2):
     total = visited_pairs(T) * FLOP_PER_PAIR
     full_s = t_comp + total / rate
     return {"value": total / full_s / 1e12, "unit": "TFLOP/s", "cores": n, "kind": "oracle",
-            "sample": f"{len(starts)} groups of 128 consecutive positions spread over T={T} "
+            "sample": ("" if vha_rank is None else f"with the rank-{vha_rank} head mix: ")
+                      + f"{len(starts)} groups of 128 consecutive positions spread over T={T} "
                       f"(all 64 heads), {sum(dt for dt, _ in res):.1f} s of oracle time on "
                       f"{n} worker processes, scaled to all {visited_pairs(T)} visited pairs; "
                       f"plus the fp64 compression of all {T // BLOCK} blocks ({t_comp:.1f} s, "
                       f"one core)"}
+
+
+def _backward_worker(seed):
+    """Seconds of one fp64 oracle backward of a T = 1024 sequence (drawing
+    the inputs is not timed)."""
+    import torch
+    torch.set_num_threads(1)
+    from compressed_sliding_window_b200 import inputs as I
+    from oracle import hca_oracle as O
+    x = I.prefill_inputs(I.PrefillConfig("bwd_sample", B=1, T=1024, seed=seed))
+    dout = _f64(I.normal_bf16(seed, "dout", 1024, (64, 512))).reshape(1, 1024, 64, 512)
+    args = [_f64(x[n]) for n in ("q", "k", "v", "s", "g")]
+    t = time.perf_counter()
+    O.prefill_backward(*args, dout)
+    return time.perf_counter() - t
+
+
+def cpu_baseline_backward(T: int):
+    """Oracle TFLOP/s for the backward: every core runs the oracle backward
+    of its own T = 1024 sequence; the rate of all cores together (FLOPs of
+    the five pair-GEMMs over busy time, summed) is scaled to T."""
+    n = host_cores()
+    pool = _cpu_pool(n, None, ())
+    try:
+        res = pool.map(_backward_worker, [9700 + i for i in range(n)], chunksize=1)
+    finally:
+        pool.close()
+        pool.join()
+    flops_sample = 5 * visited_pairs(1024) * FLOP_PER_PAIR // 2
+    rate = flops_sample * n / (sum(res) / n)           # FLOP/s, all cores
+    return {"value": rate / 1e12, "unit": "TFLOP/s", "cores": n, "kind": "oracle",
+            "sample": f"{n} oracle backward passes of T=1024 sequences, one per worker process, "
+                      f"{sum(res):.1f} s of oracle time; the rate (FLOPs of the five pair-GEMMs "
+                      f"over busy time) applies to T={T} by its visited pairs"}
 
 
 def _decode_worker(job):
@@ -519,6 +555,11 @@ def run_ours(args):
             result.setdefault("side_errors", {})["backward"] = f"{type(e).__name__}: {e}"[:300]
     if rank == 0 and world == 1 and not args.no_cpu:
         result["cpu_baseline"] = cpu_baseline_prefill(cfg)
+        if not args.quick and "vha" in result:
+            result["vha"]["cpu_baseline"] = cpu_baseline_prefill(cfg, vha_rank=VHA_RANK,
+                                                                 groups_per_core=1)
+        if not args.quick and "backward" in result:
+            result["backward"]["cpu_baseline"] = cpu_baseline_backward(cfg.T)
         if not args.quick and "prefill_32k" in result:
             result["prefill_32k"]["cpu_baseline"] = cpu_baseline_prefill(I.PREFILL_32K)
         if not args.quick and "decode" in result:
