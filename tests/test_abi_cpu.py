@@ -243,3 +243,27 @@ def test_python_binding_fails_loudly_without_gpu():
     s = torch.zeros((1, 256), dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         hca.compress(x, x, s)
+
+
+def test_python_binding_checks_new_entry_points_without_gpu():
+    """The head-mix and backward bindings refuse host tensors (no CPU
+    fallback) and malformed factors before touching the library."""
+    import torch
+    import compressed_sliding_window_b200 as hca
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    T = 4
+    q = torch.zeros((1, T, 64, 512), dtype=torch.bfloat16)
+    k = torch.zeros((1, T, 512), dtype=torch.bfloat16)
+    s = torch.zeros((1, T), dtype=torch.bfloat16)
+    c = torch.zeros((1, 0, 512), dtype=torch.bfloat16)
+    lse = torch.zeros((1, T, 64), dtype=torch.float32)
+    f = torch.zeros((64, 8), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        hca.prefill(q, k, k, c, c, q, vha=(f, f))
+    with pytest.raises(ValueError):
+        hca.prefill_backward(q, k, k, s, c, c, q, q, lse, q)
+    with pytest.raises(ValueError):
+        hca.decode(q[0], c, c, torch.zeros((T, 128, 512), dtype=torch.bfloat16),
+                   torch.zeros((T, 128, 512), dtype=torch.bfloat16),
+                   torch.ones((T,), dtype=torch.int32), q[0], vha=(f, f))
