@@ -64,3 +64,17 @@ def test_backward_accounting():
     assert 5 * pairs * bench.FLOP_PER_PAIR // 2 == 5 * pairs * 64 * 512 * 2
     act = T * 64 * 512 * 2
     assert bench.backward_bytes(1, T) == 10 * act + 5 * pairs * 64 * 2 + 2 * T * 512 * 4
+
+
+def test_backward_child_failure_is_reported_not_raised_into_the_line():
+    """The backward measurement's child process, run where it cannot succeed
+    (no GPU here), surfaces as an exception naming its exit code, which the
+    parent records under side_errors instead of losing the line."""
+    import types
+    import pytest
+    import torch
+    import bench
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    with pytest.raises(RuntimeError, match="backward child exited"):
+        bench.run_backward_child(types.SimpleNamespace(side_steps=4))
